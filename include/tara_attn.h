@@ -1,0 +1,188 @@
+/*
+ * tara_attn.h -- C ABI of the TARA-biased joint self-attention forward pass.
+ *
+ * The operation (one joint self-attention layer of a reference-to-video diffusion
+ * transformer, forward only):
+ *
+ *   for every branch b, head h and query token i of the packed joint sequence,
+ *     s_ij = dot(Q[b,h,i,:], K[b,h,j,:]) * scale + bias_ij          (j over all N tokens)
+ *     O[b,h,i,:]  = sum_j softmax_j(s_ij) * V[b,h,j,:]
+ *     LSE[b,h,i]  = ln(sum_j exp(s_ij))
+ *
+ *   bias_ij = -min(strength * (max(|t_i - t_j| - window, 0) / falloff)^2, cap)
+ *               if token i is an output (TARGET) video token and token j belongs to the
+ *               selected motion (GUIDE) video
+ *               ("TARA: Native Temporal Alignment for MiniMax H3 References",
+ *                section "The temporal rule");
+ *           = m_i * ln(gain[pic_j])
+ *               if token i is a TARGET token with mask weight m_i and token j belongs to
+ *               native Picture pic_j
+ *               ("BFS H3 Reference Attention Binding (Experimental)", section "The exact rule");
+ *           = 0 for every other edge (text, audio, other videos, target->target, and every
+ *               query that is not a TARGET token; same two pages, same sections).
+ *
+ *   scale defaults to 1/sqrt(head_dim) (the score line of "The temporal rule"); the bias is
+ *   added after scaling.  LSE is the natural-log log-sum-exp of the scaled, biased logits,
+ *   the quantity the pages' FlashAttention-with-LSE backend merges ("TARA: ...", section
+ *   "Three backends").
+ *
+ * Conventions shared by every entry point:
+ *   - Status: 0 on success, a negative TARA_ERR_* code otherwise.  Every argument is checked
+ *     before anything is launched; a failed check launches nothing and writes nothing.  No
+ *     entry point exits, throws or prints.
+ *   - Ownership: the caller owns every buffer.  Device buffers are never freed or retained by
+ *     the library beyond the call.  tara_attn_forward keeps one internal per-device workspace
+ *     (tile summaries and per-key bias records, about 8 bytes per token plus 32 bytes per
+ *     128-token tile per metadata set); it is allocated with cudaMalloc the first time a
+ *     device sees a given size and reused afterwards, so the first call on a device (or with a
+ *     larger N) must not be made while a stream is being captured.
+ *   - Asynchrony: device work is enqueued on `stream` and the call returns without
+ *     synchronising.  Calls on different streams that use the same device share the
+ *     workspace and therefore must not overlap; serialise them on one stream.
+ */
+#ifndef TARA_ATTN_H_
+#define TARA_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------------------------- */
+#define TARA_OK                   0
+#define TARA_ERR_NULL            -1  /* a required pointer is NULL                          */
+#define TARA_ERR_SHAPE           -2  /* B/H/N/D inconsistent between tensors, or < 1        */
+#define TARA_ERR_DTYPE           -3  /* unknown dtype, or Q/K/V/O dtypes differ             */
+#define TARA_ERR_HEAD_DIM        -4  /* D not supported (tensor-core path: 64 or 128)       */
+#define TARA_ERR_PARAM           -5  /* window/falloff/strength/cap/gain/scale out of domain */
+#define TARA_ERR_ALIGN           -6  /* a device pointer is not 16-byte aligned             */
+#define TARA_ERR_SEGMENT         -7  /* packer: bad segment description                     */
+#define TARA_ERR_CAPACITY        -8  /* packer: output length does not match the segments   */
+#define TARA_ERR_CUDA            -9  /* a CUDA runtime/driver call failed                   */
+#define TARA_ERR_DEVICE_TIMEOUT -10  /* a kernel gave up on a bounded wait (see below)      */
+#define TARA_ERR_TOO_LARGE      -11  /* a size exceeds what an index type or buffer holds   */
+
+/* ---- token roles ---------------------------------------------------------------------- */
+/* Roles of the tokens of the packed joint sequence ("TARA: ...", opening paragraphs and
+ * "The temporal rule"; "BFS H3 Reference Attention Binding", "The exact rule").  Values
+ * above TARA_SEG_OTHER_VIDEO are treated as plain tokens (no bias) by the kernels.        */
+typedef enum {
+  TARA_SEG_TEXT        = 0,
+  TARA_SEG_PICTURE     = 1,  /* native Picture reference; pic = 1..9                       */
+  TARA_SEG_TARGET      = 2,  /* output (generated) video token                             */
+  TARA_SEG_GUIDE       = 3,  /* token of the selected motion <Video N> reference           */
+  TARA_SEG_AUDIO       = 4,  /* reference / guide audio, packed natively, never biased     */
+  TARA_SEG_OTHER_VIDEO = 5   /* native video reference that is not the motion source       */
+} tara_seg;
+
+typedef enum { TARA_BF16 = 0, TARA_FP16 = 1, TARA_FP32 = 2 } tara_dtype;
+
+/* A dense tensor [B][H][N][D], row-major and contiguous, in device memory. */
+typedef struct {
+  void*      ptr;
+  tara_dtype dtype;
+  int32_t    B, H, N, D;
+} tara_tensor;
+
+/* Per-token metadata of the packed sequence, four device arrays of length N each
+ * (structure of arrays).  batch_stride = 0: one set shared by all B branches (the CFG
+ * branches of one shot share their packing); otherwise set b starts at element
+ * b * batch_stride of every array and there are B sets.
+ *   seg    : tara_seg value per token
+ *   time_s : seconds on the shared 24 fps clock after temporal RoPE alignment (only read for
+ *            TARGET and GUIDE tokens)
+ *   pic    : Picture index 1..9 for PICTURE tokens (0 elsewhere; indices outside 1..9 are
+ *            neutral)
+ *   m      : mask weight of TARGET tokens, normally in [0,1] (a value outside is used as is) */
+typedef struct {
+  const uint8_t* seg;
+  const float*   time_s;
+  const uint8_t* pic;
+  const float*   m;
+  int32_t        N;
+  int64_t        batch_stride;
+} tara_token_meta;
+
+/* Rule parameters.  Defaults ("TARA: ...", "The temporal rule"): window 0.20 s,
+ * falloff 0.25 s, strength 2.0, cap 6.0.  gain[i-1] is the gain of Picture i
+ * ("BFS H3 Reference Attention Binding", "Inputs you'll set": reference_strength for the
+ * chosen Picture, other_reference_strength for the others, 1 = neutral).
+ * Domain: falloff > 0; window, strength, cap >= 0; gain > 0; all finite.
+ * softmax_scale: 0 selects 1/sqrt(D); otherwise a finite positive value used as is.        */
+typedef struct {
+  float window, falloff, strength, cap;
+  float gain[9];
+  float softmax_scale;
+} tara_params;
+
+/* Fill *p with the defaults above (all gains 1, softmax_scale 0).  NULL is ignored. */
+void tara_default_params(tara_params* p);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* tara_status_string(int status);
+
+/* ---- the forward pass ------------------------------------------------------------------ */
+/* Computes O and LSE as defined at the top of this file.
+ *   Q, K, V : device tensors [B][H][N][D], same shape and dtype.  bf16/fp16 run on the
+ *             tensor-core kernel (D = 64 or 128); fp32 runs on the exact CUDA-core kernel
+ *             (any D from 1 to 256).  Base pointers 16-byte aligned.
+ *   meta    : per-token metadata (device pointers), meta->N == N.
+ *   p       : rule parameters (host pointer, read during the call only).
+ *   O       : device tensor [B][H][N][D] of the same dtype (written).
+ *   LSE     : device float array [B][H][N] (written).
+ *   stream  : CUDA stream (cudaStream_t), 0 for the legacy default stream.
+ * Every O row and LSE entry is written; no other memory of the caller is touched.
+ * Errors: TARA_ERR_NULL, _SHAPE, _DTYPE, _HEAD_DIM, _PARAM, _ALIGN, _TOO_LARGE (checked
+ * before any launch), TARA_ERR_CUDA (workspace allocation or launch failure).             */
+int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
+                      const tara_token_meta* meta, const tara_params* p,
+                      tara_tensor* O, float* LSE, void* stream);
+
+/* Every kernel bounds each of its waits.  A kernel that gives up sets a per-device status
+ * word and returns early (its outputs are then unspecified).  This call synchronises
+ * `stream`, returns TARA_ERR_DEVICE_TIMEOUT if the word is set (and clears it), TARA_ERR_CUDA
+ * if the synchronisation failed, TARA_OK otherwise.                                       */
+int tara_device_status(void* stream);
+
+/* ---- the token-metadata packer (host) ------------------------------------------------- */
+/* One segment of the packed joint sequence, in packing order.  A segment is `frames` latent
+ * frames of `tokens_per_frame` tokens each (text, pictures and audio use frames = 1).
+ * Token (f, p) of a segment (frame f, patch p in row-major patch order) gets
+ *   seg    = kind
+ *   time_s = (float)(t0_s + f * frame_dt_s)       evaluated in double, rounded once
+ *   pic    = pic for PICTURE segments (must be 1..9), 0 otherwise
+ *   m      = mask value for TARGET segments: 1 if mask_len == 0 (no mask: the gain applies to
+ *            the whole output video); mask[p] if mask_len == tokens_per_frame (one static
+ *            mask); mask[f*tokens_per_frame + p] if mask_len == frames*tokens_per_frame (one
+ *            mask per frame); 1 for every non-TARGET token.
+ * ("BFS H3 Reference Attention Binding", "Inputs you'll set": no mask, one static mask, or
+ * one mask per prepared shot frame; the mask is taken here already at patch resolution.)   */
+typedef struct {
+  int32_t      kind;              /* tara_seg                                               */
+  int32_t      frames;            /* >= 1                                                   */
+  int32_t      tokens_per_frame;  /* >= 1                                                   */
+  int32_t      pic;               /* PICTURE: 1..9; ignored otherwise                       */
+  double       t0_s;              /* time of frame 0 on the shared clock                    */
+  double       frame_dt_s;        /* seconds per latent frame (e.g. 4/24)                   */
+  const float* mask;              /* host array, TARGET only; may be NULL if mask_len == 0  */
+  int64_t      mask_len;
+} tara_segment;
+
+/* Total token count of a segment list (>= 0), or a negative status on a bad list. */
+int64_t tara_packed_length(const tara_segment* segs, int32_t n_segs);
+
+/* Write the four metadata arrays (host memory, capacity N each) for the segment list.
+ * Returns TARA_ERR_NULL, TARA_ERR_SEGMENT (kind > 5, frames or tokens_per_frame < 1, PICTURE
+ * without pic in 1..9, mask_len not in {0, tokens_per_frame, frames*tokens_per_frame}, or a
+ * non-finite time), TARA_ERR_CAPACITY (N != total length) or TARA_OK.  Nothing is written
+ * unless the whole list is valid.                                                         */
+int tara_pack_token_meta(const tara_segment* segs, int32_t n_segs,
+                         uint8_t* seg, float* time_s, uint8_t* pic, float* m, int32_t N);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TARA_ATTN_H_ */
