@@ -1,0 +1,190 @@
+"""The C ABI on the host (no GPU): exports, argument checks, and the token packer.
+
+Every call to tara_attn_forward here fails its argument checks before anything touches a
+device, so the fake pointers below are never dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from video_diffusion_attention_b200 import _binding as B
+from video_diffusion_attention_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return B.load_library()
+
+
+def declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names.update(re.findall(r"\b(tara_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert {"tara_attn_forward", "tara_pack_token_meta", "tara_default_params"} <= names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(B.EXPORTS) <= names
+
+
+def test_status_strings(lib):
+    for code in list(B.STATUS) + [-99]:
+        assert lib.tara_status_string(code)
+
+
+def test_default_params_are_the_pages_defaults(lib, golden_rule):
+    p = B.default_params()
+    for key in ("window", "falloff", "strength", "cap"):
+        assert getattr(p, key) == pytest.approx(golden_rule[key][0], rel=1e-7)
+    assert list(p.gain) == [1.0] * 9 and p.softmax_scale == 0.0
+
+
+# ---------------------------------------------------------------------------------------
+# argument checks (fake, never-dereferenced pointers)
+# ---------------------------------------------------------------------------------------
+FAKE = 0x7f0000001000
+
+
+def _t(ptr=FAKE, dtype=B.TARA_BF16, shape=(1, 2, 300, 128)):
+    t = B.TaraTensor()
+    t.ptr, t.dtype = ptr, dtype
+    t.B, t.H, t.N, t.D = shape
+    return t
+
+
+def _meta(N=300, stride=0, ptr=FAKE):
+    m = B.TaraTokenMeta()
+    m.seg = m.pic = ptr
+    m.time_s = m.m = ptr
+    m.N, m.batch_stride = N, stride
+    return m
+
+
+def _call(lib, Q=None, K=None, V=None, meta=None, p=None, O=None, lse=FAKE):
+    Q, K, V, O = (x if x is not None else _t() for x in (Q, K, V, O))
+    meta = meta if meta is not None else _meta()
+    p = p if p is not None else B.make_params()
+    return lib.tara_attn_forward(ctypes.byref(Q), ctypes.byref(K), ctypes.byref(V),
+                                 ctypes.byref(meta), ctypes.byref(p), ctypes.byref(O),
+                                 ctypes.c_void_p(lse), None)
+
+
+def test_rejects_null(lib):
+    assert lib.tara_attn_forward(None, None, None, None, None, None, None, None) == -1
+    assert _call(lib, Q=_t(ptr=0)) == -1
+    assert _call(lib, lse=0) == -1
+    assert _call(lib, meta=_meta(ptr=0)) == -1
+
+
+def test_rejects_dtype(lib):
+    assert _call(lib, K=_t(dtype=B.TARA_FP16)) == -3
+    assert _call(lib, O=_t(dtype=B.TARA_FP32)) == -3
+    assert _call(lib, Q=_t(dtype=7), K=_t(dtype=7), V=_t(dtype=7), O=_t(dtype=7)) == -3
+
+
+def test_rejects_shape(lib):
+    assert _call(lib, K=_t(shape=(1, 2, 299, 128))) == -2
+    assert _call(lib, V=_t(shape=(1, 3, 300, 128))) == -2
+    assert _call(lib, O=_t(shape=(2, 2, 300, 128))) == -2
+    assert _call(lib, meta=_meta(N=301)) == -2
+    assert _call(lib, meta=_meta(stride=10)) == -2
+    assert _call(lib, meta=_meta(stride=-1)) == -2
+    z = (1, 2, 0, 128)
+    assert _call(lib, Q=_t(shape=z), K=_t(shape=z), V=_t(shape=z), O=_t(shape=z),
+                 meta=_meta(N=0)) == -2
+
+
+def test_rejects_head_dim(lib):
+    for d in (32, 96, 256):
+        s = (1, 2, 300, d)
+        assert _call(lib, Q=_t(shape=s), K=_t(shape=s), V=_t(shape=s), O=_t(shape=s)) == -4
+    s = (1, 2, 300, 257)
+    f = B.TARA_FP32
+    assert _call(lib, Q=_t(dtype=f, shape=s), K=_t(dtype=f, shape=s), V=_t(dtype=f, shape=s),
+                 O=_t(dtype=f, shape=s)) == -4
+
+
+def test_rejects_misalignment(lib):
+    assert _call(lib, V=_t(ptr=FAKE + 8)) == -6
+    assert _call(lib, lse=FAKE + 2) == -6
+
+
+@pytest.mark.parametrize("kw", [
+    dict(falloff=0.0), dict(falloff=-1.0), dict(window=-0.1), dict(strength=-2.0),
+    dict(cap=-1.0), dict(cap=float("inf")), dict(window=float("nan")),
+    dict(gain=(0.0,) + (1.0,) * 8), dict(gain=(1.0,) * 8 + (-1.0,)),
+    dict(gain=(float("inf"),) + (1.0,) * 8), dict(softmax_scale=-1.0),
+])
+def test_rejects_parameters(lib, kw):
+    assert _call(lib, p=B.make_params(**kw)) == -5
+
+
+# ---------------------------------------------------------------------------------------
+# the packer against the oracle's packer (bit-exact) and its error handling
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("name", W.ORDER)
+def test_packer_matches_oracle_bit_exact(lib, name):
+    segs = W.get(name).segments
+    a = B.pack_token_meta(segs)
+    b = oracle.pack_token_meta(segs)
+    assert B.packed_length(segs) == len(b["seg"])
+    for key in ("seg", "time_s", "pic", "m"):
+        np.testing.assert_array_equal(a[key].view(np.uint8), b[key].view(np.uint8))
+
+
+def test_packer_mask_modes_and_offsets(lib):
+    rng = np.random.Generator(np.random.PCG64(5))
+    segs = [
+        W.Segment(W.TARGET, 3, 7, t0_s=0.25, frame_dt_s=1 / 24, mask=rng.uniform(0, 1, 7).astype(np.float32)),
+        W.Segment(W.TARGET, 3, 7, t0_s=-1.0, frame_dt_s=4 / 24, mask=rng.uniform(0, 1, 21).astype(np.float32)),
+        W.Segment(W.TARGET, 2, 5),
+        W.Segment(W.GUIDE, 4, 3, t0_s=1 / 24, frame_dt_s=4 / 24),
+        W.Segment(W.PICTURE, 1, 4, pic=9),
+        W.Segment(W.OTHER_VIDEO, 2, 2, frame_dt_s=0.5),
+    ]
+    a = B.pack_token_meta(segs)
+    b = oracle.pack_token_meta(segs)
+    for key in ("seg", "time_s", "pic", "m"):
+        np.testing.assert_array_equal(a[key].view(np.uint8), b[key].view(np.uint8))
+
+
+@pytest.mark.parametrize("bad", [
+    W.Segment(9, 1, 4),
+    W.Segment(W.TEXT, 0, 4),
+    W.Segment(W.TEXT, 1, 0),
+    W.Segment(W.PICTURE, 1, 4, pic=0),
+    W.Segment(W.PICTURE, 1, 4, pic=10),
+    W.Segment(W.TARGET, 2, 4, mask=np.ones(5, np.float32)),
+    W.Segment(W.GUIDE, 2, 4, mask=np.ones(4, np.float32)),
+    W.Segment(W.TARGET, 2, 4, t0_s=float("nan")),
+])
+def test_packer_rejects_bad_segments(lib, bad):
+    with pytest.raises(B.TaraError) as e:
+        B.pack_token_meta([W.Segment(W.TEXT, 1, 3), bad])
+    assert e.value.code == -7
+
+
+def test_packer_capacity_mismatch(lib):
+    arr, keep = B._segments_to_c([W.Segment(W.TEXT, 1, 10)])
+    buf = np.zeros(64, np.uint8)
+    fb = np.zeros(64, np.float32)
+    rc = lib.tara_pack_token_meta(arr, 1, buf.ctypes.data, fb.ctypes.data, buf.ctypes.data,
+                                  fb.ctypes.data, 11)
+    assert rc == -8
+    assert lib.tara_pack_token_meta(arr, 1, None, None, None, None, 10) == -1

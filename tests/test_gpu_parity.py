@@ -1,0 +1,150 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from parity_util import TOL, compare, rows_from_sample, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _check(w, rows=None, per_branch_meta=False, seed_device=DEV):
+    q, k, v = W.make_qkv(w, seed_device)
+    q, k, v = q.to(DEV), k.to(DEV), v.to(DEV)
+    O, L = run_gpu(w, q, k, v, per_branch_meta=per_branch_meta)
+    if rows is None:
+        rows = oracle.all_rows(w.B, w.H, w.N)
+    Oref, Lref = run_oracle(w, q, k, v, rows)
+    return compare(w, O, L, rows, Oref, Lref, w.dtype)
+
+
+# ---------------------------------------------------------------------------------------
+# the five workloads
+# ---------------------------------------------------------------------------------------
+def test_tiny_fp32_all_rows():
+    _check(W.get("tiny"))
+
+
+def test_medium_bf16_all_rows():
+    _check(W.get("medium"))
+
+
+@pytest.mark.parametrize("name", ["micro", "full", "ragged"])
+def test_large_sampled_rows(name):
+    w = W.get(name)
+    _check(w, rows_from_sample(W.sample_rows(w, per_head=256)))
+
+
+def test_ragged_per_branch_metadata():
+    # the same packing supplied once per CFG branch (batch-strided metadata)
+    w = W.get("ragged")
+    rows = rows_from_sample({k: v[:64] for k, v in W.sample_rows(w, per_head=64).items()
+                             if k[1] < 4})
+    _check(w, rows, per_branch_meta=True)
+
+
+# ---------------------------------------------------------------------------------------
+# dtypes and head dims
+# ---------------------------------------------------------------------------------------
+def _small(name, dtype, D, segs, params=None, H=2, B=1, qk=1.0, seed=200):
+    return W.custom(name, B=B, H=H, D=D, dtype=dtype, segments=segs, params=params,
+                    qk_scale=qk, seed_index=seed)
+
+
+def _layout(tpf=40, frames=5, guide_t0=0.0, picture=(96, 1)):
+    return [
+        W.Segment(W.TEXT, 1, 37),
+        W.Segment(W.PICTURE, 1, picture[0], pic=picture[1]),
+        W.Segment(W.TARGET, frames, tpf, frame_dt_s=4 / 24,
+                  mask=W.uniform_mask(7, tpf)),
+        W.Segment(W.GUIDE, frames, tpf, t0_s=guide_t0, frame_dt_s=4 / 24),
+        W.Segment(W.AUDIO, 1, 21),
+    ]
+
+
+GAINS = W.Params(gain=(1.25, 0.75) + (1.0,) * 7)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_dtype_headdim(dtype, D):
+    w = _small("dt", dtype, D, _layout(tpf=64, frames=7), GAINS, H=3)
+    _check(w)
+
+
+def test_fp32_head_dim_128_and_odd():
+    _check(_small("f32a", "fp32", 128, _layout(tpf=24, frames=6), GAINS))
+    _check(_small("f32b", "fp32", 72, _layout(tpf=10, frames=6), GAINS))
+
+
+# ---------------------------------------------------------------------------------------
+# edge cases: sizes, tails, roles, parameters
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("N", [1, 2, 31, 127, 128, 129, 255, 257, 383])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_ragged_lengths(N, dtype):
+    # one target frame block and one guide block split around the middle; plain text pads
+    nt = N // 3
+    ng = N // 3
+    segs = [W.Segment(W.TEXT, 1, N - nt - ng)] if N - nt - ng > 0 else []
+    if nt:
+        segs.append(W.Segment(W.TARGET, 1, nt, frame_dt_s=4 / 24))
+    if ng:
+        segs.append(W.Segment(W.GUIDE, 1, ng, t0_s=0.5))
+    D = 128 if dtype == "bf16" else 64
+    _check(_small("len%d" % N, dtype, D, segs, W.Params(), H=2, seed=300 + N))
+
+
+def test_no_target_rows_is_plain_attention():
+    segs = [W.Segment(W.TEXT, 1, 200), W.Segment(W.GUIDE, 3, 50, frame_dt_s=0.2),
+            W.Segment(W.PICTURE, 1, 60, pic=1)]
+    _check(_small("notgt", "bf16", 128, segs, GAINS))
+
+
+def test_every_tile_class():
+    # constant-cap tiles (distant frames), constant-picture tiles (a long single picture),
+    # zero tiles (near frames, no gain) and per-edge tiles (boundaries) in one call
+    segs = [
+        W.Segment(W.TEXT, 1, 64),
+        W.Segment(W.PICTURE, 1, 384, pic=1),
+        W.Segment(W.PICTURE, 1, 256, pic=2),
+        W.Segment(W.TARGET, 10, 128, frame_dt_s=4 / 24, mask=W.uniform_mask(9, 128)),
+        W.Segment(W.GUIDE, 10, 128, frame_dt_s=4 / 24),
+        W.Segment(W.AUDIO, 1, 100),
+    ]
+    _check(_small("cls", "bf16", 128, segs, GAINS, H=2, qk=1.5))
+
+
+@pytest.mark.parametrize("p", [
+    W.Params(strength=0.0),
+    W.Params(cap=0.0),
+    W.Params(window=0.0, falloff=0.05, strength=5.0, cap=12.0),
+    W.Params(window=1.0),
+    W.Params(gain=(3.0,) + (0.2,) * 8),
+    W.Params(softmax_scale=0.05),
+])
+def test_parameter_corners(p):
+    _check(_small("par", "bf16", 128, _layout(tpf=50, frames=8), p, H=2))
+
+
+def test_unsorted_roles_and_other_video():
+    # roles interleaved out of the usual order, plus a non-selected video reference
+    segs = [
+        W.Segment(W.GUIDE, 2, 70, t0_s=0.3, frame_dt_s=4 / 24),
+        W.Segment(W.TARGET, 3, 45, frame_dt_s=4 / 24),
+        W.Segment(W.PICTURE, 1, 33, pic=3),
+        W.Segment(W.OTHER_VIDEO, 2, 40, frame_dt_s=4 / 24),
+        W.Segment(W.TARGET, 2, 45, t0_s=0.5, frame_dt_s=4 / 24),
+        W.Segment(W.TEXT, 1, 9),
+    ]
+    _check(_small("mix", "bf16", 128, segs, W.Params(gain=(1.0, 1.0, 2.0) + (1.0,) * 6)))
+
+
+def test_batch_of_branches_shared_and_strided_meta():
+    w = _small("br", "bf16", 128, _layout(tpf=40, frames=4), GAINS, H=2, B=3)
+    _check(w)
+    _check(w, per_branch_meta=True)

@@ -1,0 +1,231 @@
+"""ctypes binding of libtara_attn.so (argument marshalling only).
+
+Every step of the attention runs in the library's kernels; this module only turns torch
+tensors and Python segment lists into the C structs of include/tara_attn.h.  There is no
+fallback: if the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libtara_attn.so")
+
+TARA_BF16, TARA_FP16, TARA_FP32 = 0, 1, 2
+SEG_TEXT, SEG_PICTURE, SEG_TARGET, SEG_GUIDE, SEG_AUDIO, SEG_OTHER_VIDEO = range(6)
+
+STATUS = {
+    0: "TARA_OK", -1: "TARA_ERR_NULL", -2: "TARA_ERR_SHAPE", -3: "TARA_ERR_DTYPE",
+    -4: "TARA_ERR_HEAD_DIM", -5: "TARA_ERR_PARAM", -6: "TARA_ERR_ALIGN",
+    -7: "TARA_ERR_SEGMENT", -8: "TARA_ERR_CAPACITY", -9: "TARA_ERR_CUDA",
+    -10: "TARA_ERR_DEVICE_TIMEOUT", -11: "TARA_ERR_TOO_LARGE",
+}
+EXPORTS = ("tara_default_params", "tara_status_string", "tara_attn_forward",
+           "tara_device_status", "tara_packed_length", "tara_pack_token_meta")
+
+
+class TaraError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s (%d)" % (what, STATUS.get(code, "?"), code))
+        self.code = code
+
+
+class TaraTensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("dtype", ctypes.c_int), ("B", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("D", ctypes.c_int32)]
+
+
+class TaraTokenMeta(ctypes.Structure):
+    _fields_ = [("seg", ctypes.c_void_p), ("time_s", ctypes.c_void_p),
+                ("pic", ctypes.c_void_p), ("m", ctypes.c_void_p), ("N", ctypes.c_int32),
+                ("batch_stride", ctypes.c_int64)]
+
+
+class TaraParams(ctypes.Structure):
+    _fields_ = [("window", ctypes.c_float), ("falloff", ctypes.c_float),
+                ("strength", ctypes.c_float), ("cap", ctypes.c_float),
+                ("gain", ctypes.c_float * 9), ("softmax_scale", ctypes.c_float)]
+
+
+class TaraSegment(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("frames", ctypes.c_int32),
+                ("tokens_per_frame", ctypes.c_int32), ("pic", ctypes.c_int32),
+                ("t0_s", ctypes.c_double), ("frame_dt_s", ctypes.c_double),
+                ("mask", ctypes.c_void_p), ("mask_len", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load_library(path: Optional[str] = None):
+    """Load the library (once).  Raises OSError when it is missing: there is no fallback."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise OSError("libtara_attn.so not built (%s); run "
+                      "`python -m video_diffusion_attention_b200.build`" % p)
+    lib = ctypes.CDLL(p)
+    lib.tara_default_params.restype = None
+    lib.tara_default_params.argtypes = [ctypes.POINTER(TaraParams)]
+    lib.tara_status_string.restype = ctypes.c_char_p
+    lib.tara_status_string.argtypes = [ctypes.c_int]
+    lib.tara_attn_forward.restype = ctypes.c_int
+    lib.tara_attn_forward.argtypes = [ctypes.POINTER(TaraTensor)] * 3 + [
+        ctypes.POINTER(TaraTokenMeta), ctypes.POINTER(TaraParams), ctypes.POINTER(TaraTensor),
+        ctypes.c_void_p, ctypes.c_void_p]
+    lib.tara_device_status.restype = ctypes.c_int
+    lib.tara_device_status.argtypes = [ctypes.c_void_p]
+    lib.tara_packed_length.restype = ctypes.c_int64
+    lib.tara_packed_length.argtypes = [ctypes.POINTER(TaraSegment), ctypes.c_int32]
+    lib.tara_pack_token_meta.restype = ctypes.c_int
+    lib.tara_pack_token_meta.argtypes = [ctypes.POINTER(TaraSegment), ctypes.c_int32] + [
+        ctypes.c_void_p] * 4 + [ctypes.c_int32]
+    if path is None:
+        _lib = lib
+    return lib
+
+
+# ---------------------------------------------------------------------------------------
+# parameters and packing
+# ---------------------------------------------------------------------------------------
+def make_params(window=0.20, falloff=0.25, strength=2.0, cap=6.0, gain=(1.0,) * 9,
+                softmax_scale=0.0) -> TaraParams:
+    p = TaraParams()
+    p.window, p.falloff, p.strength, p.cap = window, falloff, strength, cap
+    g = list(gain)
+    if len(g) != 9:
+        raise ValueError("gain needs 9 entries (Pictures 1..9)")
+    for i in range(9):
+        p.gain[i] = g[i]
+    p.softmax_scale = softmax_scale
+    return p
+
+
+def params_from(obj) -> TaraParams:
+    """TaraParams from any object with window, falloff, strength, cap, gain, softmax_scale."""
+    return make_params(obj.window, obj.falloff, obj.strength, obj.cap, obj.gain,
+                       getattr(obj, "softmax_scale", 0.0))
+
+
+def default_params() -> TaraParams:
+    p = TaraParams()
+    load_library().tara_default_params(ctypes.byref(p))
+    return p
+
+
+def _segments_to_c(segments):
+    arr = (TaraSegment * max(1, len(segments)))()
+    keep = []
+    for i, s in enumerate(segments):
+        c = arr[i]
+        c.kind, c.frames, c.tokens_per_frame = int(s.kind), int(s.frames), int(s.tokens_per_frame)
+        c.pic = int(getattr(s, "pic", 0))
+        c.t0_s, c.frame_dt_s = float(getattr(s, "t0_s", 0.0)), float(getattr(s, "frame_dt_s", 0.0))
+        mask = getattr(s, "mask", None)
+        if mask is not None and len(mask) > 0:
+            mk = np.ascontiguousarray(mask, dtype=np.float32)
+            keep.append(mk)
+            c.mask, c.mask_len = mk.ctypes.data, mk.size
+        else:
+            c.mask, c.mask_len = None, 0
+    return arr, keep
+
+
+def packed_length(segments) -> int:
+    arr, _keep = _segments_to_c(segments)
+    n = load_library().tara_packed_length(arr, len(segments))
+    if n < 0:
+        raise TaraError(int(n), "tara_packed_length")
+    return int(n)
+
+
+def pack_token_meta(segments):
+    """Host packer: dict of numpy arrays seg (u8), time_s (f32), pic (u8), m (f32)."""
+    lib = load_library()
+    arr, _keep = _segments_to_c(segments)
+    n = lib.tara_packed_length(arr, len(segments))
+    if n < 0:
+        raise TaraError(int(n), "tara_packed_length")
+    out = {"seg": np.empty(n, np.uint8), "time_s": np.empty(n, np.float32),
+           "pic": np.empty(n, np.uint8), "m": np.empty(n, np.float32)}
+    rc = lib.tara_pack_token_meta(arr, len(segments), out["seg"].ctypes.data,
+                                  out["time_s"].ctypes.data, out["pic"].ctypes.data,
+                                  out["m"].ctypes.data, int(n))
+    if rc != 0:
+        raise TaraError(rc, "tara_pack_token_meta")
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# device calls (torch tensors in, torch tensors out)
+# ---------------------------------------------------------------------------------------
+class DeviceMeta:
+    """Per-token metadata resident on a device (the four arrays of tara_token_meta)."""
+
+    def __init__(self, meta: dict, device, batch_stride: int = 0, N: Optional[int] = None):
+        import torch
+        self.seg = torch.as_tensor(np.ascontiguousarray(meta["seg"]), dtype=torch.uint8).to(device)
+        self.time_s = torch.as_tensor(np.ascontiguousarray(meta["time_s"]),
+                                      dtype=torch.float32).to(device)
+        self.pic = torch.as_tensor(np.ascontiguousarray(meta["pic"]), dtype=torch.uint8).to(device)
+        self.m = torch.as_tensor(np.ascontiguousarray(meta["m"]), dtype=torch.float32).to(device)
+        self.batch_stride = int(batch_stride)
+        self.N = int(self.seg.numel()) if N is None else int(N)
+
+    def c_struct(self, N: Optional[int] = None) -> TaraTokenMeta:
+        c = TaraTokenMeta()
+        c.seg, c.time_s = self.seg.data_ptr(), self.time_s.data_ptr()
+        c.pic, c.m = self.pic.data_ptr(), self.m.data_ptr()
+        c.N = self.N if N is None else N
+        c.batch_stride = self.batch_stride
+        return c
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.bfloat16: TARA_BF16, torch.float16: TARA_FP16, torch.float32: TARA_FP32}[t.dtype]
+
+
+def tensor_struct(t) -> TaraTensor:
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous [B][H][N][D]")
+    c = TaraTensor()
+    c.ptr = t.data_ptr()
+    c.dtype = _dtype_code(t)
+    c.B, c.H, c.N, c.D = (int(x) for x in t.shape)
+    return c
+
+
+def attn_forward(q, k, v, meta: DeviceMeta, params: TaraParams, out=None, lse=None,
+                 stream=None):
+    """O, LSE = the TARA-biased attention forward of q, k, v ([B][H][N][D] CUDA tensors)."""
+    import torch
+    lib = load_library()
+    B, H, N, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    cq, ck, cv, co = tensor_struct(q), tensor_struct(k), tensor_struct(v), tensor_struct(out)
+    cm = meta.c_struct()
+    rc = lib.tara_attn_forward(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv),
+                               ctypes.byref(cm), ctypes.byref(params), ctypes.byref(co),
+                               ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise TaraError(rc, "tara_attn_forward")
+    return out, lse
+
+
+def device_status(stream=None) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(load_library().tara_device_status(ctypes.c_void_p(stream.cuda_stream)))

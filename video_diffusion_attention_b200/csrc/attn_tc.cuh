@@ -1,0 +1,383 @@
+// attn_tc.cuh -- the tensor-core path: one-pass TARA-biased attention forward on sm_100a.
+//
+// One CTA owns two 128-row query tiles of one (branch, head) and streams every 128-key tile
+// of K and V once.  Warp roles (384 threads):
+//   warps 0-3  softmax for query tile 0   (thread = one query row = one TMEM lane)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q once, then K_j, V_j into a ring of shared-memory slots
+//   warp  9    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j with tcgen05.mma;
+//              also owns the tensor-memory allocation
+//   warps 10-11 idle (complete the third warpgroup for the register split)
+// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1, fp32.  P_t (16-bit) is written by the
+// softmax threads into columns 64..127 of S_t and read from there as the A operand of the PV
+// MMA, so P never goes through shared memory.
+//
+// The bias never exists as an N x N tensor.  For each (query tile, key tile) pair the softmax
+// warps classify the pair from the two tile summaries: no bias, a constant -cap on every
+// target row, a constant m_row*ln(gain) on every target row, or per-edge evaluation from the
+// per-key records.  Constant biases fold into the per-row exponent offset, so they cost no
+// per-element work.  Logits are kept in log2 units: x = s*scale*log2(e) + bias*log2(e).
+//
+// Online softmax: a thread holds its whole row of S (32x32b TMEM loads give one row per
+// thread), so the row max and sum need no cross-thread reduction.  The running max is only
+// raised when it grows by more than 2^8 in weight (P stays below 256), and only then is the
+// O row in TMEM rescaled, after the previous PV MMA has completed.
+#pragma once
+
+#include "sm100_ptx.cuh"
+#include "tara_common.cuh"
+
+namespace tara {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait; a normal wait is microseconds
+constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s to let in-flight copies/MMAs land
+
+template <int D>
+struct TcShape {
+  static constexpr int kTileBytes = kTile * D * 2;          // one 128 x D 16-bit tile
+  static constexpr int kPanels = D / 64;                    // 128-byte swizzle panels per row
+  static constexpr int kPanelBytes = kTile * 128;           // 128 rows x 128 bytes
+  static constexpr int kStages = (D == 128) ? 4 : 8;        // K/V ring slots
+  static constexpr int kBarCount = 1 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kSmemBytes =
+      1024 /*alignment slack*/ + 2 * kTileBytes + kStages * kTileBytes + kBarCount * 8 + 16;
+  static constexpr uint32_t kColS = 0;        // S_t at kColS + 128 t
+  static constexpr uint32_t kColO = 256;      // O_t at kColO + D t
+  static constexpr uint32_t kColP = 64;       // P_t at S_t + kColP
+};
+
+struct TcArgs {
+  void* O;
+  float* LSE;
+  const uint8_t* seg;
+  const float* time_s;
+  const float* m;
+  const TileRec* recs;
+  const float2* keyinfo;
+  long long meta_stride;   // tokens between metadata sets (0: one set for all branches)
+  int N, H, ntiles;
+  int per_branch_meta;     // 1 when every branch has its own metadata set
+  int* status;
+  BiasParams bp;
+};
+
+// A wait every lane of the warp leaves together (the tcgen05 loads and stores that follow are
+// warp-collective).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <bool kBF16>
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+  return kBF16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
+}
+
+template <bool kBF16, int D>
+__global__ void __launch_bounds__(384, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const TcArgs args) {
+  using S = TcShape<D>;
+  constexpr int TB = S::kTileBytes;
+  constexpr int NS = S::kStages;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                       // 2 tiles
+  uint8_t* sKV = smem + 2 * TB;             // NS slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * TB);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + NS;
+  uint64_t* s_full = kv_empty + NS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* drain = pv_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = args.N;
+  const int bh = blockIdx.z * args.H + blockIdx.y;
+  const int qt0 = blockIdx.x * 2;
+  const int nk = (N + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&pv_done[t], 1);
+    }
+    mbar_init(drain, 1);
+    // a CTA that starts after another one gave up does no work at all
+    *abort_flag = (*reinterpret_cast<volatile int*>(args.status) != 0) ? 1 : 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (*abort_flag) return;
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory");
+    if (warp == 8 && lane == 0) {
+      // ------------------------------ TMA producer ------------------------------
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(q_full, 2 * TB);
+      for (int t = 0; t < 2; ++t)
+        for (int p = 0; p < S::kPanels; ++p)
+          tma_load_3d(sQ + t * TB + p * S::kPanelBytes, &tmQ, q_full, p * 64, (qt0 + t) * kTile, bh);
+      int issued = 0;
+      for (int i = 0; i < 2 * nk; ++i) {
+        const int slot = i % NS;
+        const uint32_t ph = (uint32_t)(i / NS) & 1u;
+        if (!mbar_wait(&kv_empty[slot], ph ^ 1u, abort_flag, kWaitLimitNs)) break;
+        mbar_arrive_expect_tx(&kv_full[slot], TB);
+        const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+        for (int p = 0; p < S::kPanels; ++p)
+          tma_load_3d(sKV + slot * TB + p * S::kPanelBytes, map, &kv_full[slot], p * 64,
+                      (i >> 1) * kTile, bh);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        // let the copies already issued land before the CTA's shared memory is released
+        volatile int no_abort = 0;
+        mbar_wait(q_full, 0, &no_abort, kDrainLimitNs);
+        for (int i = issued - NS < 0 ? 0 : issued - NS; i < issued; ++i)
+          mbar_wait(&kv_full[i % NS], (uint32_t)(i / NS) & 1u, &no_abort, kDrainLimitNs);
+      }
+    } else if (warp == 9 && lane == 0) {
+      // ------------------------------ MMA issuer --------------------------------
+      constexpr uint32_t idesc_qk = make_idesc_f16(128, 128, kBF16, false);
+      constexpr uint32_t idesc_pv = make_idesc_f16(128, D, kBF16, true);
+      const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
+      bool ok = mbar_wait(q_full, 0, abort_flag, kWaitLimitNs);
+      tc_fence_after();
+      for (int j = 0; ok && j <= nk; ++j) {
+        const int ki = 2 * j, kslot = ki % NS;
+        if (j < nk) {
+          if (!(ok = mbar_wait(&kv_full[kslot], (uint32_t)(ki / NS) & 1u, abort_flag, kWaitLimitNs))) break;
+          tc_fence_after();
+        }
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j > 0) {
+            const int vi = 2 * (j - 1) + 1, vslot = vi % NS;
+            if (t == 0) {
+              if (!(ok = mbar_wait(&kv_full[vslot], (uint32_t)(vi / NS) & 1u, abort_flag, kWaitLimitNs))) break;
+            }
+            if (!(ok = mbar_wait(&p_full[t], (uint32_t)(j - 1) & 1u, abort_flag, kWaitLimitNs))) break;
+            tc_fence_after();
+            const uint32_t d_o = tmem + S::kColO + t * D;
+            const uint32_t a_p = tmem + S::kColS + t * 128 + S::kColP;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t bdesc = make_sdesc_sw128(sKVa + vslot * TB + kk * 2048, S::kPanelBytes, 1024);
+              umma_ts(d_o, a_p + kk * 8, bdesc, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&pv_done[t]);
+            if (t == 1) umma_commit(&kv_empty[vslot]);
+          }
+          if (j < nk) {
+            const uint32_t d_s = tmem + S::kColS + t * 128;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * S::kPanelBytes + (kk & 3) * 32;
+              const uint64_t adesc = make_sdesc_sw128(sQa + t * TB + off, 16, 1024);
+              const uint64_t bdesc = make_sdesc_sw128(sKVa + kslot * TB + off, 16, 1024);
+              umma_ss(d_s, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[t]);
+            if (t == 1) umma_commit(&kv_empty[kslot]);
+          }
+        }
+      }
+      // every MMA issued above completes before tensor memory is released
+      umma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort, kDrainLimitNs);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;\n" ::: "memory");
+    // ------------------------------ softmax warps -------------------------------
+    const int t = warp >> 2;            // query tile of this warpgroup
+    const int wq = warp & 3;            // TMEM lane quarter
+    const int r = wq * 32 + lane;       // row within the tile
+    const int qtile = qt0 + t;
+    const int row = qtile * kTile + r;
+    const bool row_ok = (qtile < args.ntiles) && (row < N);
+    const BiasParams& bp = args.bp;
+    const int mset = args.per_branch_meta ? blockIdx.z : 0;
+    const long long mtok = (long long)mset * args.meta_stride;
+    const TileRec* recs = args.recs + (long long)mset * args.ntiles;
+    const float2* kinfo = args.keyinfo + (long long)mset * N;
+
+    bool is_tgt = false;
+    float t_q = 0.0f, m_q = 0.0f;
+    if (row_ok) {
+      is_tgt = args.seg[mtok + row] == kSegTarget;
+      t_q = args.time_s[mtok + row];
+      m_q = args.m[mtok + row];
+    }
+    TileRec qr;
+    if (qtile < args.ntiles) {
+      qr = recs[qtile];
+    } else {
+      qr.segmask = 0;
+      qr.picmask = 0;
+      qr.nvalid = 0;
+      qr.single_pic = 0;
+      qr.tq_min = qr.tk_min = 0.0f;
+      qr.tq_max = qr.tk_max = 0.0f;
+    }
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + S::kColS + t * 128;
+    const uint32_t tP = tS + S::kColP;
+    const uint32_t tO = tmem + lane_off + S::kColO + t * D;
+    const float ninf = __int_as_float(0xff800000);
+    float m_run = ninf, l_run = 0.0f;
+    bool ok = true;
+
+    for (int j = 0; j < nk; ++j) {
+      const TileRec kr = recs[j];
+      float cval;
+      const int cls = classify_pair(qr, kr, bp, &cval);
+      float rowb2 = 0.0f;
+      if (is_tgt) {
+        if (cls == kClsConstCap) rowb2 = cval * kLog2e;
+        else if (cls == kClsConstPic) rowb2 = (m_q * cval) * kLog2e;
+      }
+      if (!(ok = warp_wait(&s_full[t], (uint32_t)j & 1u, abort_flag, kWaitLimitNs))) break;
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_ld_wait();
+      reg_fence<128>(s);
+      const int nv = (int)kr.nvalid;
+      if (nv < kTile) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= nv) s[c] = 0xff800000u;
+      }
+      float mx, scl, off_base;
+      if (cls == kClsFull) {
+        const float2* kp = kinfo + (long long)j * kTile;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float2 ki = kp[c < nv ? c : 0];
+          const float b = is_tgt ? edge_bias_target(t_q, m_q, __float_as_int(ki.x), ki.y, bp) : 0.0f;
+          s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), bp.scale_log2, b * kLog2e));
+        }
+        float a0 = ninf, a1 = ninf;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          a0 = fmaxf(a0, __uint_as_float(s[c]));
+          a1 = fmaxf(a1, __uint_as_float(s[c + 1]));
+        }
+        mx = fmaxf(a0, a1);
+        scl = 1.0f;
+        off_base = 0.0f;
+      } else {
+        float a0 = ninf, a1 = ninf;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          a0 = fmaxf(a0, __uint_as_float(s[c]));
+          a1 = fmaxf(a1, __uint_as_float(s[c + 1]));
+        }
+        mx = fmaf(fmaxf(a0, a1), bp.scale_log2, rowb2);
+        scl = bp.scale_log2;
+        off_base = rowb2;
+      }
+      const float m_new = fmaxf(m_run, mx);
+      const bool need = (m_new - m_run) > 8.0f;        // true on the first tile (m_run = -inf)
+      const float m_use = need ? m_new : m_run;
+      const float alpha = ex2_approx(m_run - m_use);   // 1 when not raised, 0 on the first tile
+      l_run *= alpha;
+      const float off = off_base - m_use;
+      uint32_t pk[64];
+      float l0 = 0.0f, l1 = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), scl, off));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), scl, off));
+        l0 += p0;
+        l1 += p1;
+        pk[c >> 1] = pack_p<kBF16>(p0, p1);
+      }
+      l_run += l0 + l1;
+      tmem_st32(tP + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // rescale this warp's O rows once the previous PV has landed
+        if (!(ok = warp_wait(&pv_done[t], (uint32_t)(j - 1) & 1u, abort_flag, kWaitLimitNs))) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait();
+          reg_fence<32>(o);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(tO + cc * 32, o);
+        }
+      }
+      m_run = m_use;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    // ------------------------------ epilogue ---------------------------------------
+    if (ok && warp_wait(&pv_done[t], (uint32_t)(nk - 1) & 1u, abort_flag, kWaitLimitNs)) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l_run;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(args.O) + ((long long)bh * N + row) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_ld_wait();
+        reg_fence<32>(o);
+        if (row_ok) {
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_p<kBF16>(__uint_as_float(o[2 * c]) * inv_l,
+                                 __uint_as_float(o[2 * c + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+      if (row_ok) args.LSE[(long long)bh * N + row] = (m_run + log2f(l_run)) * kLn2;
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(args.status, 1);
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace tara

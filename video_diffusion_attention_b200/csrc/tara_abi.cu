@@ -1,0 +1,298 @@
+// tara_abi.cu -- the C ABI of the library: argument checks, the per-device workspace, tensor
+// maps, and the launches of the tile-summary, tensor-core and CUDA-core kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "tara_attn.h"
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+#include "tile_summary.cuh"
+
+namespace tara {
+namespace {
+
+// Set by any kernel that gave up on a bounded wait; read and cleared by tara_device_status.
+__device__ int g_device_status;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  void* ws = nullptr;           // tile summaries + per-key records
+  size_t ws_bytes = 0;
+  int* status = nullptr;        // device address of g_device_status
+  bool tc_attr_set[2][2] = {{false, false}, {false, false}};   // [bf16][D==128]
+  bool simt_attr_set = false;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int get_encode_fn() {
+  if (g_encode) return TARA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                       &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return TARA_ERR_CUDA;
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return TARA_OK;
+}
+
+bool finite_f(float x) { return std::isfinite(x); }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_params(const tara_params* p) {
+  if (!finite_f(p->window) || !finite_f(p->falloff) || !finite_f(p->strength) ||
+      !finite_f(p->cap) || !finite_f(p->softmax_scale))
+    return TARA_ERR_PARAM;
+  if (p->falloff <= 0.0f || p->window < 0.0f || p->strength < 0.0f || p->cap < 0.0f ||
+      p->softmax_scale < 0.0f)
+    return TARA_ERR_PARAM;
+  for (int i = 0; i < 9; ++i)
+    if (!finite_f(p->gain[i]) || p->gain[i] <= 0.0f) return TARA_ERR_PARAM;
+  return TARA_OK;
+}
+
+BiasParams make_bias_params(const tara_params* p, int D) {
+  BiasParams bp;
+  std::memset(&bp, 0, sizeof(bp));
+  bp.window = p->window;
+  bp.inv_falloff = (float)(1.0 / (double)p->falloff);
+  bp.strength = p->strength;
+  bp.cap = p->cap;
+  const double scale = p->softmax_scale > 0.0f ? (double)p->softmax_scale
+                                                : 1.0 / std::sqrt((double)D);
+  bp.scale = (float)scale;
+  bp.scale_log2 = (float)(scale * 1.4426950408889634);
+  bp.lng_nz = 0;
+  for (int i = 1; i <= 9; ++i) {
+    bp.lng[i] = (float)std::log((double)p->gain[i - 1]);
+    if (bp.lng[i] != 0.0f) bp.lng_nz |= 1u << i;
+  }
+  return bp;
+}
+
+int encode_qkv_map(CUtensorMap* map, const tara_tensor* t) {
+  const CUtensorMapDataType dt =
+      t->dtype == TARA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t dims[3] = {(cuuint64_t)t->D, (cuuint64_t)t->N,
+                              (cuuint64_t)t->B * (cuuint64_t)t->H};
+  const cuuint64_t strides[2] = {(cuuint64_t)t->D * 2, (cuuint64_t)t->N * (cuuint64_t)t->D * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, dt, 3, t->ptr, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TARA_OK : TARA_ERR_CUDA;
+}
+
+// Returns the device's state with a workspace of at least `bytes` (grown with cudaMalloc).
+int device_state(size_t bytes, DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TARA_ERR_CUDA;
+  DeviceState& st = g_dev[dev];
+  if (st.status == nullptr) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return TARA_ERR_CUDA;
+    st.status = static_cast<int*>(addr);
+  }
+  if (bytes > st.ws_bytes) {
+    if (st.ws) {
+      cudaFree(st.ws);   // synchronises the device: no earlier call still reads it
+      st.ws = nullptr;
+      st.ws_bytes = 0;
+    }
+    if (cudaMalloc(&st.ws, bytes) != cudaSuccess) {
+      st.ws = nullptr;
+      return TARA_ERR_CUDA;
+    }
+    st.ws_bytes = bytes;
+  }
+  *out = &st;
+  return TARA_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+template <bool kBF16, int D>
+int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+              const TcArgs& a, int B, int H, int ntiles, cudaStream_t stream, DeviceState* st) {
+  constexpr int smem = TcShape<D>::kSmemBytes;
+  bool& attr = st->tc_attr_set[kBF16 ? 1 : 0][D == 128 ? 1 : 0];
+  if (!attr) {
+    if (cudaFuncSetAttribute(attn_tc_kernel<kBF16, D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return TARA_ERR_CUDA;
+    attr = true;
+  }
+  dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
+  attn_tc_kernel<kBF16, D><<<grid, 384, smem, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
+}
+
+int validate(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
+             const tara_token_meta* meta, const tara_params* p, const tara_tensor* O,
+             const float* LSE) {
+  if (!Q || !K || !V || !meta || !p || !O || !LSE) return TARA_ERR_NULL;
+  if (!Q->ptr || !K->ptr || !V->ptr || !O->ptr) return TARA_ERR_NULL;
+  if (!meta->seg || !meta->time_s || !meta->pic || !meta->m) return TARA_ERR_NULL;
+  const tara_tensor* ts[4] = {Q, K, V, O};
+  for (const tara_tensor* t : ts) {
+    if (t->dtype != TARA_BF16 && t->dtype != TARA_FP16 && t->dtype != TARA_FP32)
+      return TARA_ERR_DTYPE;
+    if (t->dtype != Q->dtype) return TARA_ERR_DTYPE;
+    if (t->B < 1 || t->H < 1 || t->N < 1 || t->D < 1) return TARA_ERR_SHAPE;
+    if (t->B != Q->B || t->H != Q->H || t->N != Q->N || t->D != Q->D) return TARA_ERR_SHAPE;
+  }
+  if (meta->N != Q->N) return TARA_ERR_SHAPE;
+  if (meta->batch_stride < 0 || (meta->batch_stride != 0 && meta->batch_stride < meta->N))
+    return TARA_ERR_SHAPE;
+  if (Q->dtype == TARA_FP32) {
+    if (Q->D > kSimtMaxD) return TARA_ERR_HEAD_DIM;
+  } else {
+    if (Q->D != 64 && Q->D != 128) return TARA_ERR_HEAD_DIM;
+  }
+  if (Q->B > 65535 || Q->H > 65535) return TARA_ERR_TOO_LARGE;
+  if ((long long)Q->B * Q->H > 0x7fffffffLL) return TARA_ERR_TOO_LARGE;
+  for (const tara_tensor* t : ts)
+    if (!aligned16(t->ptr)) return TARA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(LSE) & 3u) != 0) return TARA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(meta->time_s) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(meta->m) & 3u) != 0)
+    return TARA_ERR_ALIGN;
+  return check_params(p);
+}
+
+}  // namespace
+}  // namespace tara
+
+using namespace tara;
+
+extern "C" {
+
+void tara_default_params(tara_params* p) {
+  if (!p) return;
+  p->window = 0.20f;
+  p->falloff = 0.25f;
+  p->strength = 2.0f;
+  p->cap = 6.0f;
+  for (int i = 0; i < 9; ++i) p->gain[i] = 1.0f;
+  p->softmax_scale = 0.0f;
+}
+
+const char* tara_status_string(int s) {
+  switch (s) {
+    case TARA_OK: return "ok";
+    case TARA_ERR_NULL: return "null pointer";
+    case TARA_ERR_SHAPE: return "inconsistent or invalid shape";
+    case TARA_ERR_DTYPE: return "invalid or mismatched dtype";
+    case TARA_ERR_HEAD_DIM: return "unsupported head dimension";
+    case TARA_ERR_PARAM: return "rule parameter out of domain";
+    case TARA_ERR_ALIGN: return "misaligned pointer";
+    case TARA_ERR_SEGMENT: return "invalid segment description";
+    case TARA_ERR_CAPACITY: return "output length does not match the segments";
+    case TARA_ERR_CUDA: return "CUDA call failed";
+    case TARA_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case TARA_ERR_TOO_LARGE: return "size too large";
+    default: return "unknown status";
+  }
+}
+
+int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
+                      const tara_token_meta* meta, const tara_params* p, tara_tensor* O,
+                      float* LSE, void* stream_) {
+  int rc = validate(Q, K, V, meta, p, O, LSE);
+  if (rc != TARA_OK) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
+  const BiasParams bp = make_bias_params(p, D);
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (Q->dtype == TARA_FP32) {
+    DeviceState* st = nullptr;
+    if ((rc = device_state(0, &st)) != TARA_OK) return rc;
+    const size_t smem = (size_t)(2 * kSimtChunk * (D + 1) + kSimtRows * D) * sizeof(float);
+    if (!st->simt_attr_set) {
+      if (cudaFuncSetAttribute(attn_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)((2 * kSimtChunk * (kSimtMaxD + 1) + kSimtRows * kSimtMaxD) *
+                                     sizeof(float))) != cudaSuccess)
+        return TARA_ERR_CUDA;
+      st->simt_attr_set = true;
+    }
+    dim3 grid((unsigned)((N + kSimtRows - 1) / kSimtRows), (unsigned)H, (unsigned)B);
+    attn_simt_kernel<<<grid, kSimtRows * 32, smem, stream>>>(
+        static_cast<const float*>(Q->ptr), static_cast<const float*>(K->ptr),
+        static_cast<const float*>(V->ptr), static_cast<float*>(O->ptr), LSE, meta->seg,
+        meta->time_s, meta->pic, meta->m, (long long)meta->batch_stride, H, N, D, bp);
+    return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
+  }
+
+  if ((rc = get_encode_fn()) != TARA_OK) return rc;
+  const int ntiles = (N + kTile - 1) / kTile;
+  const int nsets = meta->batch_stride != 0 ? B : 1;
+  const size_t rec_bytes = round_up((size_t)nsets * ntiles * sizeof(TileRec), 256);
+  const size_t key_bytes = round_up((size_t)nsets * N * sizeof(float2), 256);
+  DeviceState* st = nullptr;
+  if ((rc = device_state(rec_bytes + key_bytes, &st)) != TARA_OK) return rc;
+  TileRec* recs = static_cast<TileRec*>(st->ws);
+  float2* keyinfo = reinterpret_cast<float2*>(static_cast<char*>(st->ws) + rec_bytes);
+
+  CUtensorMap mq, mk, mv;
+  if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K) != TARA_OK ||
+      encode_qkv_map(&mv, V) != TARA_OK)
+    return TARA_ERR_CUDA;
+
+  tile_summary_kernel<<<dim3((unsigned)ntiles, (unsigned)nsets), 128, 0, stream>>>(
+      meta->seg, meta->time_s, meta->pic, N, (long long)meta->batch_stride, ntiles, bp, recs,
+      keyinfo);
+  if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
+
+  TcArgs a;
+  a.O = O->ptr;
+  a.LSE = LSE;
+  a.seg = meta->seg;
+  a.time_s = meta->time_s;
+  a.m = meta->m;
+  a.recs = recs;
+  a.keyinfo = keyinfo;
+  a.meta_stride = (long long)meta->batch_stride;
+  a.N = N;
+  a.H = H;
+  a.ntiles = ntiles;
+  a.per_branch_meta = meta->batch_stride != 0 ? 1 : 0;
+  a.status = st->status;
+  a.bp = bp;
+  const bool bf16 = Q->dtype == TARA_BF16;
+  if (D == 128)
+    return bf16 ? launch_tc<true, 128>(mq, mk, mv, a, B, H, ntiles, stream, st)
+                : launch_tc<false, 128>(mq, mk, mv, a, B, H, ntiles, stream, st);
+  return bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
+              : launch_tc<false, 64>(mq, mk, mv, a, B, H, ntiles, stream, st);
+}
+
+int tara_device_status(void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TARA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return TARA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return TARA_ERR_CUDA;
+    return TARA_ERR_DEVICE_TIMEOUT;
+  }
+  return TARA_OK;
+}
+
+}  // extern "C"
