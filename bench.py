@@ -1,0 +1,384 @@
+"""Benchmark of the TARA-biased joint attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full] [--impl ours|reference]
+
+One step = one call of tara_attn_forward (tile summaries + the attention kernel) over the
+workload's whole batch, inputs resident in HBM.  The default workload is the 56-head,
+107,126-token bf16 shot with reference binding (Q/K/V/O 6.1 GB, far above the 126 MB L2, so
+no L2 flush is needed between steps).  With --gpus N > 1 (torchrun), every rank runs its own
+replica of the workload with no collective on the data path (weak scaling); the time is the
+max over ranks.  Prints one JSON line on rank 0.
+
+--impl reference times the fp64 CPU oracle instead, on bounded row samples of the same
+workload (the pages ship no code to run, so the oracle is the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_tc_dram_traffic.txt")
+CSRC = os.path.join(ROOT, "video_diffusion_attention_b200", "csrc")
+
+
+def describe(w: W.Workload) -> dict:
+    segs = []
+    names = {0: "text", 1: "picture", 2: "target", 3: "guide", 4: "audio", 5: "other_video"}
+    for s in w.segments:
+        d = {"role": names[s.kind], "tokens": s.length}
+        if s.frames > 1:
+            d["frames"] = s.frames
+        segs.append(d)
+    return {"workload": "%s: B=%d H=%d N=%d D=%d %s" % (w.name, w.B, w.H, w.N, w.D, w.dtype),
+            "B": w.B, "H": w.H, "N": w.N, "head_dim": w.D, "segments": segs,
+            "params": {"window": w.params.window, "falloff": w.params.falloff,
+                       "strength": w.params.strength, "cap": w.params.cap,
+                       "gain": list(w.params.gain)},
+            "flop_per_step": w.flops,
+            "l2": "inputs %.1f GB > 126 MB L2; no flush" % (4 * w.B * w.H * w.N * w.D * 2 / 1e9)}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary, if it was
+    taken on the current kernel source; None otherwise."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    vals = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if "=" in line:
+                k, v = line.split("=", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    key = "bytes_per_launch_" + workload
+    return float(vals[key]) if key in vals else None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.device_index)
+            bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", bus, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        under_load = [x for x in sm if x > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(under_load) if under_load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample_rate(w: W.Workload, budget_s: float, device_inputs=None, seed: int = 11):
+    """Time the oracle on seeded query rows of workload w for about budget_s seconds.
+
+    Returns (rows, seconds, threads).  Inputs are the workload's own seeded tensors (drawn on
+    the GPU when one is given, else on the CPU)."""
+    import torch
+    import oracle
+    if device_inputs is not None:
+        q, k, v = device_inputs
+    else:
+        q, k, v = W.make_qkv(w, "cpu")
+    raw = [oracle.torch_to_numpy_raw(t) for t in (q, k, v)]
+    meta = oracle.pack_token_meta(w.segments)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    threads = oracle.max_threads()
+
+    def run(n):
+        rows = np.stack([rng.integers(0, w.B, n), rng.integers(0, w.H, n),
+                         rng.integers(0, w.N, n)], axis=1).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention_rows(raw[0][0], raw[1][0], raw[2][0], raw[0][1], meta, w.params, rows)
+        return time.perf_counter() - t0
+
+    probe = max(threads, 16)
+    dt = run(probe)
+    n = max(probe, int(probe * budget_s / max(dt, 1e-6)))
+    dt = run(n)
+    return n, dt, threads
+
+
+def run_reference(args, w: W.Workload):
+    """The oracle arm: K timed steps, each a bounded row sample of the workload."""
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    q, k, v = W.make_qkv(w, "cpu")
+    raw = [oracle.torch_to_numpy_raw(t) for t in (q, k, v)]
+    meta = oracle.pack_token_meta(w.segments)
+    threads = oracle.max_threads()
+    rng = np.random.Generator(np.random.PCG64(5))
+    flop_per_row = 4.0 * w.N * w.D
+    # size one step at about 8 s of CPU work
+    probe = max(16, threads)
+    rows = np.stack([rng.integers(0, w.B, probe), rng.integers(0, w.H, probe),
+                     rng.integers(0, w.N, probe)], axis=1).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.attention_rows(raw[0][0], raw[1][0], raw[2][0], raw[0][1], meta, w.params, rows)
+    per_row = (time.perf_counter() - t0) / probe
+    n = max(threads, int(8.0 / max(per_row, 1e-9)))
+    times = []
+    for step in range(args.warmup + args.steps):
+        rows = np.stack([rng.integers(0, w.B, n), rng.integers(0, w.H, n),
+                         rng.integers(0, w.N, n)], axis=1).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention_rows(raw[0][0], raw[1][0], raw[2][0], raw[0][1], meta, w.params, rows)
+        if step >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = n * len(times) * flop_per_row / total / 1e12
+    sample = "%d random query rows per step of %s (each row: all %d keys, fp64)" % (n, w.name, w.N)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": describe(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+METRIC = "biased-attn fwd TFLOP/s at 107,126 tok bf16; % of B200 dense-BF16 peak"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="full", choices=W.ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = W.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+
+    import torch
+    import torch.distributed as dist
+    import video_diffusion_attention_b200 as T
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    lib = T.load_library()   # raises if the CUDA library is missing: no fallback
+    q, k, v = W.make_qkv(w, dev)
+    meta = T.DeviceMeta(T.pack_token_meta(w.segments), dev)
+    params = T.params_from(w.params)
+    O = torch.empty_like(q)
+    L = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        T.attn_forward(q, k, v, meta, params, O, L, stream)
+    torch.cuda.synchronize(dev)
+    if T.device_status() != 0:
+        raise SystemExit("kernel reported a device timeout during warm-up")
+
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in kev:   # create the events' handles; the library re-records them per call
+        a.record(stream)
+        b.record(stream)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(args.steps):
+        T.set_kernel_events(*kev[i])
+        T.attn_forward(q, k, v, meta, params, O, L, stream)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    if T.device_status() != 0:
+        raise SystemExit("kernel reported a device timeout in the timed region")
+    ms_total = start.elapsed_time(stop)
+    kernel_ms = [a.elapsed_time(b) for a, b in kev]
+    if world > 1:
+        t = torch.tensor([ms_total, statistics.mean(kernel_ms)], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, kmean = float(t[0]), float(t[1])
+    else:
+        kmean = statistics.mean(kernel_ms)
+    ms_step = ms_total / args.steps
+    value = world * w.flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the C ABI with host buffers: H2D of Q/K/V and metadata, the forward,
+    # D2H of O and LSE, every step, all inside the timed region
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hmeta = {key: getattr(meta, key).cpu().pin_memory() for key in ("seg", "time_s", "pic", "m")}
+    hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    hL = torch.empty(L.shape, dtype=L.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dmeta = T.DeviceMeta({kk: vv.numpy() for kk, vv in hmeta.items()}, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + sum(
+        t.numel() * t.element_size() for t in hmeta.values())
+    d2h = hO.numel() * hO.element_size() + hL.numel() * hL.element_size()
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        for key in ("seg", "time_s", "pic", "m"):
+            getattr(dmeta, key).copy_(hmeta[key], non_blocking=True)
+        T.attn_forward(dq, dk, dv, dmeta, params, O, L, stream)
+        hO.copy_(O, non_blocking=True)
+        hL.copy_(L, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = world * w.flops / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    achieved = w.flops / (kmean * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops_sustained"])
+    traffic = recorded_traffic(w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Q/K/V ~ N(0,1), packed shot layout; no dataset or weights)",
+        "config": describe(w),
+        "pct_of_dense_bf16_peak": {
+            "sustained_measured": 100.0 * value / world / float(peaks["bf16_tflops_sustained"]),
+            "burst_measured": 100.0 * value / world / float(peaks["bf16_tflops"]),
+            "nominal_2250": 100.0 * value / world / 2250.0, "peaks_source": peak_src},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "attn_tc_kernel", "kernel_ms": kmean,
+                     "peak_kind": "bf16_tflops_sustained (%s): the kernel runs back to back for "
+                                  "seconds" % peak_src},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, dt, threads = oracle_sample_rate(w, args.cpu_budget, device_inputs=(q, k, v))
+        line["cpu_baseline"] = {
+            "value": n * 4.0 * w.N * w.D / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": "%d seeded query rows of %s in %.1f s (each row against all %d keys, "
+                      "fp64)" % (n, w.name, dt, w.N)}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

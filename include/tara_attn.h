@@ -140,6 +140,13 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
                       const tara_token_meta* meta, const tara_params* p,
                       tara_tensor* O, float* LSE, void* stream);
 
+/* Profiling hook: the next tara_attn_forward call made by this host thread records the CUDA
+ * event `start` on its stream immediately before launching its attention kernel and `stop`
+ * immediately after it (the tile-summary kernel is outside the pair).  Both are cudaEvent_t
+ * handles created by the caller; NULL for both clears a pending pair.  The pair is used once.
+ * Returns TARA_OK, or TARA_ERR_NULL when exactly one of the two is NULL.                   */
+int tara_set_kernel_events(void* start, void* stop);
+
 /* Every kernel bounds each of its waits.  A kernel that gives up sets a per-device status
  * word and returns early (its outputs are then unspecified).  This call synchronises
  * `stream`, returns TARA_ERR_DEVICE_TIMEOUT if the word is set (and clears it), TARA_ERR_CUDA

@@ -25,7 +25,8 @@ STATUS = {
     -10: "TARA_ERR_DEVICE_TIMEOUT", -11: "TARA_ERR_TOO_LARGE",
 }
 EXPORTS = ("tara_default_params", "tara_status_string", "tara_attn_forward",
-           "tara_device_status", "tara_packed_length", "tara_pack_token_meta")
+           "tara_device_status", "tara_packed_length", "tara_pack_token_meta",
+           "tara_set_kernel_events")
 
 
 class TaraError(RuntimeError):
@@ -79,6 +80,8 @@ def load_library(path: Optional[str] = None):
     lib.tara_attn_forward.argtypes = [ctypes.POINTER(TaraTensor)] * 3 + [
         ctypes.POINTER(TaraTokenMeta), ctypes.POINTER(TaraParams), ctypes.POINTER(TaraTensor),
         ctypes.c_void_p, ctypes.c_void_p]
+    lib.tara_set_kernel_events.restype = ctypes.c_int
+    lib.tara_set_kernel_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.tara_device_status.restype = ctypes.c_int
     lib.tara_device_status.argtypes = [ctypes.c_void_p]
     lib.tara_packed_length.restype = ctypes.c_int64
@@ -222,6 +225,19 @@ def attn_forward(q, k, v, meta: DeviceMeta, params: TaraParams, out=None, lse=No
     if rc != 0:
         raise TaraError(rc, "tara_attn_forward")
     return out, lse
+
+
+def set_kernel_events(start, stop) -> None:
+    """Record torch.cuda.Event `start`/`stop` around the attention kernel of the next call.
+
+    torch creates an event's handle on its first record(), so record both once beforehand."""
+    if start is not None and (start.cuda_event == 0 or stop.cuda_event == 0):
+        raise ValueError("record both events once before handing them to the library")
+    rc = load_library().tara_set_kernel_events(
+        ctypes.c_void_p(start.cuda_event if start is not None else 0),
+        ctypes.c_void_p(stop.cuda_event if stop is not None else 0))
+    if rc != 0:
+        raise TaraError(rc, "tara_set_kernel_events")
 
 
 def device_status(stream=None) -> int:

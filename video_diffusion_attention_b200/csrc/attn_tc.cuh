@@ -29,6 +29,13 @@
 
 namespace tara {
 
+// One pair of exponentials in every kExpEmuPeriod is evaluated with exp2_poly on the FMA pipe
+// instead of MUFU (0 disables the split).
+#ifndef TARA_EXP_EMU_PERIOD
+#define TARA_EXP_EMU_PERIOD 0
+#endif
+constexpr int kExpEmuPeriod = TARA_EXP_EMU_PERIOD;
+
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait; a normal wait is microseconds
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s to let in-flight copies/MMAs land
 
@@ -38,9 +45,10 @@ struct TcShape {
   static constexpr int kPanels = D / 64;                    // 128-byte swizzle panels per row
   static constexpr int kPanelBytes = kTile * 128;           // 128 rows x 128 bytes
   static constexpr int kStages = (D == 128) ? 4 : 8;        // K/V ring slots
+  static constexpr int kKeyBufBytes = 2 * 2 * kTile * 16;  // [query tile][parity][key] float4
   static constexpr int kBarCount = 1 + 2 * kStages + 2 + 2 + 2 + 1;
-  static constexpr int kSmemBytes =
-      1024 /*alignment slack*/ + 2 * kTileBytes + kStages * kTileBytes + kBarCount * 8 + 16;
+  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + 2 * kTileBytes +
+                                    kStages * kTileBytes + kKeyBufBytes + kBarCount * 8 + 16;
   static constexpr uint32_t kColS = 0;        // S_t at kColS + 128 t
   static constexpr uint32_t kColO = 256;      // O_t at kColO + D t
   static constexpr uint32_t kColP = 64;       // P_t at S_t + kColP
@@ -53,7 +61,7 @@ struct TcArgs {
   const float* time_s;
   const float* m;
   const TileRec* recs;
-  const float2* keyinfo;
+  const float4* keyinfo;
   long long meta_stride;   // tokens between metadata sets (0: one set for all branches)
   int N, H, ntiles;
   int per_branch_meta;     // 1 when every branch has its own metadata set
@@ -67,6 +75,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
                                           uint64_t limit_ns) {
   const bool ok = mbar_wait(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
+}
+
+// Max of the 128 values of a row, as eight independent chains and a final tree.
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(s[i]);
+#pragma unroll
+  for (int c = 8; c < 128; ++c) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(s[c]));
+  return fmaxf(fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])),
+               fmaxf(fmaxf(a[4], a[5]), fmaxf(a[6], a[7])));
 }
 
 template <bool kBF16>
@@ -87,7 +106,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                       // 2 tiles
   uint8_t* sKV = smem + 2 * TB;             // NS slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * TB);
+  float4* kbuf = reinterpret_cast<float4*>(sKV + NS * TB);    // per-key records of full tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * TB + S::kKeyBufBytes);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + NS;
@@ -132,7 +152,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 152;\n" ::: "memory");
     if (warp == 8 && lane == 0) {
       // ------------------------------ TMA producer ------------------------------
       tma_prefetch_desc(&tmQ);
@@ -212,7 +232,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_wait(drain, 0, &no_abort, kDrainLimitNs);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;\n" ::: "memory");
     // ------------------------------ softmax warps -------------------------------
     const int t = warp >> 2;            // query tile of this warpgroup
     const int wq = warp & 3;            // TMEM lane quarter
@@ -224,7 +244,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int mset = args.per_branch_meta ? blockIdx.z : 0;
     const long long mtok = (long long)mset * args.meta_stride;
     const TileRec* recs = args.recs + (long long)mset * args.ntiles;
-    const float2* kinfo = args.keyinfo + (long long)mset * N;
+    const float4* kinfo = args.keyinfo + (long long)mset * N;
 
     bool is_tgt = false;
     float t_q = 0.0f, m_q = 0.0f;
@@ -252,14 +272,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float m_run = ninf, l_run = 0.0f;
     bool ok = true;
 
+    TileRec kr_next = recs[0];
     for (int j = 0; j < nk; ++j) {
-      const TileRec kr = recs[j];
+      const TileRec kr = kr_next;
+      if (j + 1 < nk) kr_next = recs[j + 1];   // in flight while this tile is processed
       float cval;
       const int cls = classify_pair(qr, kr, bp, &cval);
       float rowb2 = 0.0f;
       if (is_tgt) {
         if (cls == kClsConstCap) rowb2 = cval * kLog2e;
         else if (cls == kClsConstPic) rowb2 = (m_q * cval) * kLog2e;
+      }
+      float4* kb = kbuf + (t * 2 + (j & 1)) * kTile;
+      if (cls == kClsFull) {
+        // stage the tile's key records in shared memory (one coalesced load per thread, in
+        // flight while S is computed); two buffers, so a warp one iteration ahead never
+        // overwrites records another warp of the group still reads
+        const int key = j * kTile + r;
+        kb[r] = key < N ? kinfo[key] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        named_bar_sync(1 + t, 128);
       }
       if (!(ok = warp_wait(&s_full[t], (uint32_t)j & 1u, abort_flag, kWaitLimitNs))) break;
       tc_fence_after();
@@ -278,30 +309,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       float mx, scl, off_base;
       if (cls == kClsFull) {
-        const float2* kp = kinfo + (long long)j * kTile;
+        // branch-free per-edge bias: computed for every row, zeroed by a select on non-target
+        // rows (a per-element branch on the row role costs ~10x here)
+        const float w = bp.window, inv_f = bp.inv_falloff, st = bp.strength, cap = bp.cap;
+        const float sl = bp.scale_log2;
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
-          const float2 ki = kp[c < nv ? c : 0];
-          const float b = is_tgt ? edge_bias_target(t_q, m_q, __float_as_int(ki.x), ki.y, bp) : 0.0f;
-          s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), bp.scale_log2, b * kLog2e));
+          const float4 kv = kb[c];
+          const float x = fmaxf(fabsf(t_q - kv.x) - w, 0.0f) * inv_f;
+          const float pen = fminf(st * (x * x), cap);
+          float b = fmaf(-kv.z, pen, m_q * kv.y);
+          b = is_tgt ? b : 0.0f;
+          s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl, b * kLog2e));
         }
-        float a0 = ninf, a1 = ninf;
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          a0 = fmaxf(a0, __uint_as_float(s[c]));
-          a1 = fmaxf(a1, __uint_as_float(s[c + 1]));
-        }
-        mx = fmaxf(a0, a1);
+        mx = row_max128(s);
         scl = 1.0f;
         off_base = 0.0f;
       } else {
-        float a0 = ninf, a1 = ninf;
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          a0 = fmaxf(a0, __uint_as_float(s[c]));
-          a1 = fmaxf(a1, __uint_as_float(s[c + 1]));
-        }
-        mx = fmaf(fmaxf(a0, a1), bp.scale_log2, rowb2);
+        mx = fmaf(row_max128(s), bp.scale_log2, rowb2);
         scl = bp.scale_log2;
         off_base = rowb2;
       }
@@ -312,16 +337,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       l_run *= alpha;
       const float off = off_base - m_use;
       uint32_t pk[64];
-      float l0 = 0.0f, l1 = 0.0f;
+      float lsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
       for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), scl, off));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), scl, off));
-        l0 += p0;
-        l1 += p1;
+        // every kExpEmuPeriod-th pair of exponentials runs on the FMA pipe
+        const bool emu = kExpEmuPeriod > 0 && ((c >> 1) % (kExpEmuPeriod > 0 ? kExpEmuPeriod : 1)) ==
+                                                  (kExpEmuPeriod > 0 ? kExpEmuPeriod - 1 : 0);
+        const float x0 = fmaf(__uint_as_float(s[c]), scl, off);
+        const float x1 = fmaf(__uint_as_float(s[c + 1]), scl, off);
+        const float p0 = emu ? exp2_poly(x0) : ex2_approx(x0);
+        const float p1 = emu ? exp2_poly(x1) : ex2_approx(x1);
+        lsum[(c >> 1) & 3] += p0 + p1;
         pk[c >> 1] = pack_p<kBF16>(p0, p1);
       }
-      l_run += l0 + l1;
+      l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
       tmem_st32(tP + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       if (j > 0 && __any_sync(0xffffffffu, need)) {

@@ -217,10 +217,36 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
+// Named barrier over `count` threads (ids 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x evaluated on the FMA pipe, to take part of the exponentials off the MUFU unit.
+// Cody-Waite style split x = j + f with j = round-to-nearest(x) (|f| <= 1/2) obtained by
+// adding 1.5*2^23; 2^f from a degree-3 polynomial whose coefficients were fitted for this
+// library (relative least squares with Lawson reweighting on Chebyshev nodes of [-1/2, 1/2];
+// max relative error 7.5e-5 in fp32 Horner form, below the 2^-9 spacing of bf16); 2^j is
+// added into the exponent field.  x is clamped below at -125 (result < 2.4e-38 there).
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.055171623826026917f;
+
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(f, kExp2C3, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 }  // namespace tara

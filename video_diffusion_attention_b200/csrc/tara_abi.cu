@@ -32,6 +32,20 @@ struct DeviceState {
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 
+// Event pair set by tara_set_kernel_events for the calling thread's next forward call.
+thread_local cudaEvent_t t_ev_start = nullptr, t_ev_stop = nullptr;
+
+int record_start(cudaStream_t stream) {
+  if (t_ev_start && cudaEventRecord(t_ev_start, stream) != cudaSuccess) return TARA_ERR_CUDA;
+  return TARA_OK;
+}
+int record_stop(cudaStream_t stream) {
+  cudaEvent_t ev = t_ev_stop;
+  t_ev_start = t_ev_stop = nullptr;
+  if (ev && cudaEventRecord(ev, stream) != cudaSuccess) return TARA_ERR_CUDA;
+  return TARA_OK;
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -138,8 +152,10 @@ int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& m
     attr = true;
   }
   dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
+  if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
   attn_tc_kernel<kBF16, D><<<grid, 384, smem, stream>>>(mq, mk, mv, a);
-  return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
+  return record_stop(stream);
 }
 
 int validate(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
@@ -232,22 +248,24 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
       st->simt_attr_set = true;
     }
     dim3 grid((unsigned)((N + kSimtRows - 1) / kSimtRows), (unsigned)H, (unsigned)B);
+    if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
     attn_simt_kernel<<<grid, kSimtRows * 32, smem, stream>>>(
         static_cast<const float*>(Q->ptr), static_cast<const float*>(K->ptr),
         static_cast<const float*>(V->ptr), static_cast<float*>(O->ptr), LSE, meta->seg,
         meta->time_s, meta->pic, meta->m, (long long)meta->batch_stride, H, N, D, bp);
-    return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
+    return record_stop(stream);
   }
 
   if ((rc = get_encode_fn()) != TARA_OK) return rc;
   const int ntiles = (N + kTile - 1) / kTile;
   const int nsets = meta->batch_stride != 0 ? B : 1;
   const size_t rec_bytes = round_up((size_t)nsets * ntiles * sizeof(TileRec), 256);
-  const size_t key_bytes = round_up((size_t)nsets * N * sizeof(float2), 256);
+  const size_t key_bytes = round_up((size_t)nsets * N * sizeof(float4), 256);
   DeviceState* st = nullptr;
   if ((rc = device_state(rec_bytes + key_bytes, &st)) != TARA_OK) return rc;
   TileRec* recs = static_cast<TileRec*>(st->ws);
-  float2* keyinfo = reinterpret_cast<float2*>(static_cast<char*>(st->ws) + rec_bytes);
+  float4* keyinfo = reinterpret_cast<float4*>(static_cast<char*>(st->ws) + rec_bytes);
 
   CUtensorMap mq, mk, mv;
   if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K) != TARA_OK ||
@@ -280,6 +298,13 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
                 : launch_tc<false, 128>(mq, mk, mv, a, B, H, ntiles, stream, st);
   return bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
               : launch_tc<false, 64>(mq, mk, mv, a, B, H, ntiles, stream, st);
+}
+
+int tara_set_kernel_events(void* start, void* stop) {
+  if ((start == nullptr) != (stop == nullptr)) return TARA_ERR_NULL;
+  t_ev_start = static_cast<cudaEvent_t>(start);
+  t_ev_stop = static_cast<cudaEvent_t>(stop);
+  return TARA_OK;
 }
 
 int tara_device_status(void* stream_) {

@@ -34,9 +34,10 @@ struct __align__(16) TileRec {
   uint32_t single_pic; // p when every valid token is PICTURE with the same index p, else 0
 };
 
-// Per-key bias record: kind 0 = no bias from this key, 1 = GUIDE (value = time),
-// 2 = PICTURE with a non-neutral gain (value = ln gain).
-constexpr int kKeyPlain = 0, kKeyGuide = 1, kKeyPicture = 2;
+// Per-key bias record (float4): x = time of a GUIDE key (else 0), y = ln(gain) of a PICTURE
+// key with a non-neutral gain (else 0), z = 1 for a GUIDE key (else 0), w unused.  The bias of
+// the edge (TARGET row with time t and mask m, key) is then -z*penalty(|t - x|) + m*y, with no
+// branch on the key's role.
 
 // Tile-pair classes (per 128-row query tile x 128-key tile).
 constexpr int kClsZero = 0;      // no edge of the pair is biased
@@ -82,14 +83,6 @@ __device__ __forceinline__ int classify_pair(const TileRec& q, const TileRec& k,
     return kClsConstPic;
   }
   return kClsFull;
-}
-
-// Bias of one edge (natural units) for a TARGET query row, from the key's record.
-__device__ __forceinline__ float edge_bias_target(float t_q, float m_q, int kind, float value,
-                                                  const BiasParams& p) {
-  if (kind == kKeyGuide) return -penalty_f32(fabsf(t_q - value), p);
-  if (kind == kKeyPicture) return m_q * value;
-  return 0.0f;
 }
 
 }  // namespace tara

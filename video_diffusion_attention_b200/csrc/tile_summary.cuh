@@ -14,7 +14,7 @@ namespace tara {
 __global__ void __launch_bounds__(128)
 tile_summary_kernel(const uint8_t* __restrict__ seg, const float* __restrict__ time_s,
                     const uint8_t* __restrict__ pic, int N, long long batch_stride, int ntiles,
-                    BiasParams bp, TileRec* __restrict__ recs, float2* __restrict__ keyinfo) {
+                    BiasParams bp, TileRec* __restrict__ recs, float4* __restrict__ keyinfo) {
   const int tile = blockIdx.x;
   const int set = blockIdx.y;
   const int t = threadIdx.x;
@@ -42,18 +42,13 @@ tile_summary_kernel(const uint8_t* __restrict__ seg, const float* __restrict__ t
 
   // per-key record (the key side of the bias)
   if (valid) {
-    float2 rec;
-    int kind = kKeyPlain;
-    float value = 0.0f;
+    float4 rec = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     if (s == kSegGuide) {
-      kind = kKeyGuide;
-      value = tm;
+      rec.x = tm;
+      rec.z = 1.0f;
     } else if (s == kSegPicture && pc < 16 && bp.lng[pc] != 0.0f) {
-      kind = kKeyPicture;
-      value = bp.lng[pc];
+      rec.y = bp.lng[pc];
     }
-    rec.x = __int_as_float(kind);
-    rec.y = value;
     keyinfo[(long long)set * N + tok] = rec;
   }
 
