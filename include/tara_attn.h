@@ -140,6 +140,32 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
                       const tara_token_meta* meta, const tara_params* p,
                       tara_tensor* O, float* LSE, void* stream);
 
+/* ---- allocation-free variant ------------------------------------------------------------ */
+/* Largest scratch (bytes) tara_attn_forward_noalloc can use: per metadata set, 16 bytes per
+ * token plus 32 bytes per 128-token tile (4 MiB covers one shared set of up to ~260,000
+ * tokens).  The array is part of the loaded module: every device that loads the library
+ * holds it until the process exits.                                                       */
+#define TARA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* Same operation, arguments and checks as tara_attn_forward for bf16/fp16 inputs, but it
+ * never allocates: no cudaMalloc, no cudaFree, no allocating library call.  It is meant for
+ * callers that cannot allocate device memory while they run (work recorded into CUDA graphs,
+ * frameworks that own all device memory through their own pool, serving loops that must not
+ * stall in the allocator).  The pages have no counterpart to this entry point.
+ *   - Scratch: a fixed module array of TARA_NOALLOC_SCRATCH_BYTES on each device instead of
+ *     the cached workspace; sizes that need more return TARA_ERR_TOO_LARGE before anything
+ *     is launched.  fp32 inputs return TARA_ERR_DTYPE (their kernel needs no scratch; call
+ *     tara_attn_forward).
+ *   - Set-up: the first call on each device (that device current) looks up the array's device
+ *     address with cudaGetSymbolAddress; make that first call before any stream capture.
+ *   - Sharing: every call on a device uses the same array and leaves its contents behind;
+ *     calls never read what an earlier call left (each call rewrites every record it reads).
+ *     Calls whose work overlaps on the GPU (different streams, or concurrent with each other)
+ *     race on the array: serialise them on one stream.                                    */
+int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
+                              const tara_token_meta* meta, const tara_params* p,
+                              tara_tensor* O, float* LSE, void* stream);
+
 /* Profiling hook: the next tara_attn_forward call made by this host thread records the CUDA
  * event `start` on its stream immediately before launching its attention kernel and `stop`
  * immediately after it (the tile-summary kernel is outside the pair).  Both are cudaEvent_t

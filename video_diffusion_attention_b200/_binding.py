@@ -80,6 +80,8 @@ def load_library(path: Optional[str] = None):
     lib.tara_attn_forward.argtypes = [ctypes.POINTER(TaraTensor)] * 3 + [
         ctypes.POINTER(TaraTokenMeta), ctypes.POINTER(TaraParams), ctypes.POINTER(TaraTensor),
         ctypes.c_void_p, ctypes.c_void_p]
+    lib.tara_attn_forward_noalloc.restype = ctypes.c_int
+    lib.tara_attn_forward_noalloc.argtypes = lib.tara_attn_forward.argtypes
     lib.tara_set_kernel_events.restype = ctypes.c_int
     lib.tara_set_kernel_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.tara_device_status.restype = ctypes.c_int
@@ -238,6 +240,25 @@ def set_kernel_events(start, stop) -> None:
         ctypes.c_void_p(stop.cuda_event if stop is not None else 0))
     if rc != 0:
         raise TaraError(rc, "tara_set_kernel_events")
+
+
+def attn_forward_noalloc(q, k, v, meta: DeviceMeta, params: TaraParams, out, lse, stream=None):
+    """The same forward through tara_attn_forward_noalloc: the library allocates nothing.
+
+    `out` and `lse` must be provided by the caller (16-bit inputs only)."""
+    import torch
+    lib = load_library()
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    cq, ck, cv, co = tensor_struct(q), tensor_struct(k), tensor_struct(v), tensor_struct(out)
+    cm = meta.c_struct()
+    rc = lib.tara_attn_forward_noalloc(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv),
+                                       ctypes.byref(cm), ctypes.byref(params), ctypes.byref(co),
+                                       ctypes.c_void_p(lse.data_ptr()),
+                                       ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise TaraError(rc, "tara_attn_forward_noalloc")
+    return out, lse
 
 
 def device_status(stream=None) -> int:

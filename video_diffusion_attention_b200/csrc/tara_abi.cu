@@ -321,3 +321,125 @@ int tara_device_status(void* stream_) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of the 16-bit forward pass.
+//
+// Some callers may not allocate device memory at call time: code that records work into a
+// CUDA graph or runs under a framework's own memory pool (cudaMalloc there either fails,
+// bypasses the pool's accounting, or synchronises the device in the middle of a step), and
+// latency-bound serving loops that must never hit the driver's allocator.  For them the
+// scratch the tensor-core path needs (tile summaries and per-key bias records) lives in a
+// fixed device array that is part of the loaded module instead of the cached cudaMalloc
+// workspace used by tara_attn_forward.
+// ---------------------------------------------------------------------------------------
+namespace tara {
+namespace {
+
+constexpr size_t kStaticScratchBytes = TARA_NOALLOC_SCRATCH_BYTES;
+
+// Lives as long as the library is loaded, on every device that loads it.
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+struct StaticState {
+  bool ready = false;
+  void* scratch = nullptr;   // device address of g_static_scratch on this device
+  int* status = nullptr;     // device address of g_device_status on this device
+};
+std::mutex g_static_mu;
+StaticState g_static[kMaxDevices];
+
+// One-time set-up per device (the device must be current): device addresses of the two
+// module variables.  The host-side names of __device__ variables are stand-ins that a kernel
+// must never receive directly.
+int static_state(StaticState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TARA_ERR_CUDA;
+  StaticState& st = g_static[dev];
+  if (!st.ready) {
+    void* scratch = nullptr;
+    void* status = nullptr;
+    if (cudaGetSymbolAddress(&scratch, g_static_scratch) != cudaSuccess || scratch == nullptr)
+      return TARA_ERR_CUDA;
+    if (cudaGetSymbolAddress(&status, g_device_status) != cudaSuccess || status == nullptr)
+      return TARA_ERR_CUDA;
+    st.scratch = scratch;
+    st.status = static_cast<int*>(status);
+    st.ready = true;
+  }
+  *out = &st;
+  return TARA_OK;
+}
+
+template <bool kBF16, int D>
+int launch_tc_static(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const TcArgs& a, int B, int H, int ntiles, cudaStream_t stream) {
+  constexpr int smem = TcShape<D>::kSmemBytes;
+  if (cudaFuncSetAttribute(attn_tc_kernel<kBF16, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return TARA_ERR_CUDA;
+  dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
+  attn_tc_kernel<kBF16, D><<<grid, 384, smem, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace tara
+
+extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor* K,
+                                         const tara_tensor* V, const tara_token_meta* meta,
+                                         const tara_params* p, tara_tensor* O, float* LSE,
+                                         void* stream_) {
+  using namespace tara;
+  int rc = validate(Q, K, V, meta, p, O, LSE);
+  if (rc != TARA_OK) return rc;
+  if (Q->dtype == TARA_FP32) return TARA_ERR_DTYPE;   // the fp32 kernel needs no scratch
+  const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
+  const int ntiles = (N + kTile - 1) / kTile;
+  const size_t nsets = meta->batch_stride != 0 ? (size_t)B : 1;
+  const size_t rec_bytes = round_up(nsets * (size_t)ntiles * sizeof(TileRec), 256);
+  const size_t key_bytes = round_up(nsets * (size_t)N * sizeof(float4), 256);
+  if (rec_bytes + key_bytes > kStaticScratchBytes) return TARA_ERR_TOO_LARGE;
+
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const BiasParams bp = make_bias_params(p, D);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  StaticState* st = nullptr;
+  if ((rc = static_state(&st)) != TARA_OK) return rc;
+  if ((rc = get_encode_fn()) != TARA_OK) return rc;
+  TileRec* recs = static_cast<TileRec*>(st->scratch);
+  float4* keyinfo = reinterpret_cast<float4*>(static_cast<char*>(st->scratch) + rec_bytes);
+
+  CUtensorMap mq, mk, mv;
+  if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K) != TARA_OK ||
+      encode_qkv_map(&mv, V) != TARA_OK)
+    return TARA_ERR_CUDA;
+  // every record the attention kernel reads is rewritten here first, so the scratch needs no
+  // clearing between calls
+  tile_summary_kernel<<<dim3((unsigned)ntiles, (unsigned)nsets), 128, 0, stream>>>(
+      meta->seg, meta->time_s, meta->pic, N, (long long)meta->batch_stride, ntiles, bp, recs,
+      keyinfo);
+  if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
+
+  TcArgs a;
+  a.O = O->ptr;
+  a.LSE = LSE;
+  a.seg = meta->seg;
+  a.time_s = meta->time_s;
+  a.m = meta->m;
+  a.recs = recs;
+  a.keyinfo = keyinfo;
+  a.meta_stride = (long long)meta->batch_stride;
+  a.N = N;
+  a.H = H;
+  a.ntiles = ntiles;
+  a.per_branch_meta = meta->batch_stride != 0 ? 1 : 0;
+  a.status = st->status;
+  a.bp = bp;
+  const bool bf16 = Q->dtype == TARA_BF16;
+  if (D == 128)
+    return bf16 ? launch_tc_static<true, 128>(mq, mk, mv, a, B, H, ntiles, stream)
+                : launch_tc_static<false, 128>(mq, mk, mv, a, B, H, ntiles, stream);
+  return bf16 ? launch_tc_static<true, 64>(mq, mk, mv, a, B, H, ntiles, stream)
+              : launch_tc_static<false, 64>(mq, mk, mv, a, B, H, ntiles, stream);
+}
