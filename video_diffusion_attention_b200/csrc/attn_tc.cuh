@@ -132,7 +132,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&p_full[t], 4);   // one arrival per softmax warp
       mbar_init(&pv_done[t], 1);
     }
     mbar_init(drain, 1);
@@ -186,6 +186,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t idesc_qk = make_idesc_f16(128, 128, kBF16, false);
       constexpr uint32_t idesc_pv = make_idesc_f16(128, D, kBF16, true);
       const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
+      // base descriptors; a byte offset moves the start-address field by offset >> 4 (shared
+      // addresses stay below 2^18, so the 14-bit field never carries)
+      const uint64_t qd0 = make_sdesc_sw128(sQa, 16, 1024);
+      const uint64_t kd0 = make_sdesc_sw128(sKVa, 16, 1024);
+      const uint64_t vd0 = make_sdesc_sw128(sKVa, S::kPanelBytes, 1024);
       bool ok = mbar_wait(q_full, 0, abort_flag, kWaitLimitNs);
       tc_fence_after();
       for (int j = 0; ok && j <= nk; ++j) {
@@ -204,22 +209,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tc_fence_after();
             const uint32_t d_o = tmem + S::kColO + t * D;
             const uint32_t a_p = tmem + S::kColS + t * 128 + S::kColP;
+            const uint64_t vd = vd0 + (uint64_t)((vslot * TB) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk) {
-              const uint64_t bdesc = make_sdesc_sw128(sKVa + vslot * TB + kk * 2048, S::kPanelBytes, 1024);
-              umma_ts(d_o, a_p + kk * 8, bdesc, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              umma_ts(d_o, a_p + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                      (j > 1 || kk > 0) ? 1u : 0u);
             umma_commit(&pv_done[t]);
             if (t == 1) umma_commit(&kv_empty[vslot]);
           }
           if (j < nk) {
             const uint32_t d_s = tmem + S::kColS + t * 128;
+            const uint64_t qd = qd0 + (uint64_t)((t * TB) >> 4);
+            const uint64_t kd = kd0 + (uint64_t)((kslot * TB) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * S::kPanelBytes + (kk & 3) * 32;
-              const uint64_t adesc = make_sdesc_sw128(sQa + t * TB + off, 16, 1024);
-              const uint64_t bdesc = make_sdesc_sw128(sKVa + kslot * TB + off, 16, 1024);
-              umma_ss(d_s, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+              const uint64_t off = (uint64_t)((((kk >> 2) * S::kPanelBytes) + (kk & 3) * 32) >> 4);
+              umma_ss(d_s, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
             }
             umma_commit(&s_full[t]);
             if (t == 1) umma_commit(&kv_empty[kslot]);
@@ -332,28 +337,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       const float m_new = fmaxf(m_run, mx);
       const bool need = (m_new - m_run) > 8.0f;        // true on the first tile (m_run = -inf)
+      const bool warp_need = __any_sync(0xffffffffu, need);
       const float m_use = need ? m_new : m_run;
       const float alpha = ex2_approx(m_run - m_use);   // 1 when not raised, 0 on the first tile
       l_run *= alpha;
       const float off = off_base - m_use;
-      uint32_t pk[64];
       float lsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        // every kExpEmuPeriod-th pair of exponentials runs on the FMA pipe
-        const bool emu = kExpEmuPeriod > 0 && ((c >> 1) % (kExpEmuPeriod > 0 ? kExpEmuPeriod : 1)) ==
-                                                  (kExpEmuPeriod > 0 ? kExpEmuPeriod - 1 : 0);
-        const float x0 = fmaf(__uint_as_float(s[c]), scl, off);
-        const float x1 = fmaf(__uint_as_float(s[c + 1]), scl, off);
-        const float p0 = emu ? exp2_poly(x0) : ex2_approx(x0);
-        const float p1 = emu ? exp2_poly(x1) : ex2_approx(x1);
-        lsum[(c >> 1) & 3] += p0 + p1;
-        pk[c >> 1] = pack_p<kBF16>(p0, p1);
+      for (int half = 0; half < 2; ++half) {
+        // 64 columns at a time: their P (32 packed words) is stored while the next half runs
+        uint32_t pk[32];
+#pragma unroll
+        for (int c2 = 0; c2 < 64; c2 += 2) {
+          const int c = half * 64 + c2;
+          // every kExpEmuPeriod-th pair of exponentials runs on the FMA pipe
+          const bool emu = kExpEmuPeriod > 0 && ((c >> 1) % (kExpEmuPeriod > 0 ? kExpEmuPeriod : 1)) ==
+                                                    (kExpEmuPeriod > 0 ? kExpEmuPeriod - 1 : 0);
+          const float x0 = fmaf(__uint_as_float(s[c]), scl, off);
+          const float x1 = fmaf(__uint_as_float(s[c + 1]), scl, off);
+          const float p0 = emu ? exp2_poly(x0) : ex2_approx(x0);
+          const float p1 = emu ? exp2_poly(x1) : ex2_approx(x1);
+          lsum[(c >> 1) & 3] += p0 + p1;
+          pk[c2 >> 1] = pack_p<kBF16>(p0, p1);
+        }
+        tmem_st32(tP + half * 32, pk);
       }
       l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
-      tmem_st32(tP + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      if (j > 0 && warp_need) {
         // rescale this warp's O rows once the previous PV has landed
         if (!(ok = warp_wait(&pv_done[t], (uint32_t)(j - 1) & 1u, abort_flag, kWaitLimitNs))) break;
         tc_fence_after();
@@ -371,7 +381,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       m_run = m_use;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
 
     // ------------------------------ epilogue ---------------------------------------
