@@ -46,7 +46,7 @@ struct TcShape {
   static constexpr int kPanelBytes = kTile * 128;           // 128 rows x 128 bytes
   static constexpr int kStages = (D == 128) ? 4 : 8;        // K/V ring slots
   static constexpr int kKeyBufBytes = 2 * 2 * kTile * 16;  // [query tile][parity][key] float4
-  static constexpr int kBarCount = 1 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kBarCount = 1 + 2 * kStages + 2 + 2 + 2 + 1 + 2;
   static constexpr int kSmemBytes = 1024 /*alignment slack*/ + 2 * kTileBytes +
                                     kStages * kTileBytes + kKeyBufBytes + kBarCount * 8 + 16;
   static constexpr uint32_t kColS = 0;        // S_t at kColS + 128 t
@@ -88,6 +88,18 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
                fmaxf(fmaxf(a[4], a[5]), fmaxf(a[6], a[7])));
 }
 
+// Bounded rendezvous of the warps counted by `bar` (lane 0 of each warp arrives; every lane
+// waits).  Shared-memory writes made before it by any lane are visible to all lanes of the
+// participating warps after it.  `phase` is the caller's phase bit for this barrier.
+__device__ __forceinline__ bool warp_rendezvous(uint64_t* bar, uint32_t& phase,
+                                                volatile int* abort, uint64_t limit_ns) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = warp_wait(bar, phase, abort, limit_ns);
+  phase ^= 1u;
+  return ok;
+}
+
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
   return kBF16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
@@ -115,7 +127,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* drain = pv_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* stage_bar = drain + 1;      // [2] per query tile: the 4 warps of its group
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stage_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -136,6 +149,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&pv_done[t], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(&stage_bar[0], 4);
+    mbar_init(&stage_bar[1], 4);
     // a CTA that starts after another one gave up does no work at all
     *abort_flag = (*reinterpret_cast<volatile int*>(args.status) != 0) ? 1 : 0;
     fence_mbar_init();
@@ -277,6 +292,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float m_run = ninf, l_run = 0.0f;
     bool ok = true;
 
+    uint32_t stage_phase = 0;
     TileRec kr_next = recs[0];
     for (int j = 0; j < nk; ++j) {
       const TileRec kr = kr_next;
@@ -295,7 +311,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // overwrites records another warp of the group still reads
         const int key = j * kTile + r;
         kb[r] = key < N ? kinfo[key] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        named_bar_sync(1 + t, 128);
+        if (!(ok = warp_rendezvous(&stage_bar[t], stage_phase, abort_flag, kWaitLimitNs))) break;
       }
       if (!(ok = warp_wait(&s_full[t], (uint32_t)j & 1u, abort_flag, kWaitLimitNs))) break;
       tc_fence_after();
