@@ -189,6 +189,10 @@ def logit_row(q, k, dtype: str, meta: Dict, params, b: int, h: int, i: int,
     return out
 
 
+from .target_mask import (  # noqa: E402,F401
+    area_weights, mask_length_ok, prepare_target_mask, shot_length_ok)
+
+
 def all_rows(B: int, H: int, N: int) -> np.ndarray:
     b, h, i = np.meshgrid(np.arange(B), np.arange(H), np.arange(N), indexing="ij")
     return np.stack([b.reshape(-1), h.reshape(-1), i.reshape(-1)], axis=1).astype(np.int64)
