@@ -224,6 +224,23 @@ def run_reference(args, w: W.Workload):
 METRIC = "biased-attn fwd TFLOP/s at 107,126 tok bf16; % of B200 dense-BF16 peak"
 
 
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of a list of timings over all ranks of the default process group
+    (the slowest rank defines a multi-GPU time); identity without a group."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_throughput(flop_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own replica (weak scaling), so the job does
+    world * flop_per_rank per step in the slowest rank's step time."""
+    return world * flop_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -293,14 +310,9 @@ def main():
         raise SystemExit("kernel reported a device timeout in the timed region")
     ms_total = start.elapsed_time(stop)
     kernel_ms = [a.elapsed_time(b) for a, b in kev]
-    if world > 1:
-        t = torch.tensor([ms_total, statistics.mean(kernel_ms)], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, kmean = float(t[0]), float(t[1])
-    else:
-        kmean = statistics.mean(kernel_ms)
+    ms_total, kmean = max_over_ranks([ms_total, statistics.mean(kernel_ms)], dev)
     ms_step = ms_total / args.steps
-    value = world * w.flops / (ms_step * 1e-3) / 1e12
+    value = job_throughput(w.flops, world, ms_step)
 
     # end to end through the C ABI with host buffers: H2D of Q/K/V and metadata, the forward,
     # D2H of O and LSE, every step, all inside the timed region
@@ -335,14 +347,35 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = world * w.flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dev)[0]
+    e2e_value = job_throughput(w.flops, world, e2e_ms)
 
+    # the step before the path, measured on its own: pixel mask of a prepared 107-frame shot at
+    # 544x928 (the resolution of the pages' user run) to the workload's 26-frame target grid
+    mask_line = None
+    tgt = [sg for sg in w.segments if sg.kind == W.TARGET]
+    if tgt and tgt[0].tokens_per_frame == 2000:
+        px = torch.from_numpy(W.pixel_ellipse_mask(w.seed(3) + 1, 107, 544, 928)).to(dev)
+        mo = torch.empty((tgt[0].frames, 40, 50), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            T.prepare_target_mask(px, 107, 4, tgt[0].frames, 40, 50, out=mo, stream=stream)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        torch.cuda.synchronize(dev)
+        m0.record(stream)
+        for _ in range(reps):
+            T.prepare_target_mask(px, 107, 4, tgt[0].frames, 40, 50, out=mo, stream=stream)
+        m1.record(stream)
+        torch.cuda.synchronize(dev)
+        mms = m0.elapsed_time(m1) / reps
+        mbytes = px.numel() * 4 + mo.numel() * 4
+        mask_line = {"kernel": "target_mask_kernel", "workload": "107x544x928 fp32 pixel mask -> "
+                     "%dx40x50 target weights" % tgt[0].frames, "ms": mms, "bound": "hbm",
+                     "algorithmic_bytes": mbytes, "achieved_GBs": mbytes / (mms * 1e-3) / 1e9}
     peaks, peak_src = load_peaks()
+    if mask_line is not None:
+        mask_line["peak_GBs"] = float(peaks["hbm_gbs"])
+        mask_line["frac"] = mask_line["achieved_GBs"] / float(peaks["hbm_gbs"])
     achieved = w.flops / (kmean * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops_sustained"])
     traffic = recorded_traffic(w.name)
@@ -366,6 +399,8 @@ def main():
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
+    if mask_line is not None:
+        line["mask_prep"] = mask_line
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, dt, threads = oracle_sample_rate(w, args.cpu_budget, device_inputs=(q, k, v))
         line["cpu_baseline"] = {

@@ -63,6 +63,7 @@ extern "C" {
 #define TARA_ERR_CUDA            -9  /* a CUDA runtime/driver call failed                   */
 #define TARA_ERR_DEVICE_TIMEOUT -10  /* a kernel gave up on a bounded wait (see below)      */
 #define TARA_ERR_TOO_LARGE      -11  /* a size exceeds what an index type or buffer holds   */
+#define TARA_ERR_MASK_LENGTH    -12  /* mask neither one frame nor the 17n+5 shot length    */
 
 /* ---- token roles ---------------------------------------------------------------------- */
 /* Roles of the tokens of the packed joint sequence ("TARA: ...", opening paragraphs and
@@ -174,10 +175,43 @@ int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor* K, const 
 int tara_set_kernel_events(void* start, void* stop);
 
 /* Every kernel bounds each of its waits.  A kernel that gives up sets a per-device status
- * word and returns early (its outputs are then unspecified).  This call synchronises
+ * word and returns early (its outputs are then unspecified); while the word is set, later
+ * attention launches on that device skip their work as well.  This call synchronises
  * `stream`, returns TARA_ERR_DEVICE_TIMEOUT if the word is set (and clears it), TARA_ERR_CUDA
  * if the synchronisation failed, TARA_OK otherwise.                                       */
 int tara_device_status(void* stream);
+
+/* Self-test of that machinery (failure detection without faulting the GPU): launches one
+ * warp on `stream` that waits on a shared-memory barrier with a limit of limit_us
+ * microseconds (1..10^7).  With arrive == 0 nothing ever arrives, so the wait gives up and
+ * sets the status word, which the next tara_device_status reports; with arrive != 0 the
+ * barrier completes and nothing is set.  Returns TARA_ERR_PARAM for a limit out of range,
+ * TARA_ERR_CUDA on a launch failure, TARA_OK otherwise.  The pages have no counterpart.   */
+int tara_selftest_wait(int limit_us, int arrive, void* stream);
+
+/* ---- target-mask preparation (device) -------------------------------------------------- */
+/* Turns a soft pixel mask into the per-target-token weights m the forward pass reads
+ * ("BFS H3 Reference Attention Binding (Experimental)", "The exact rule": soft masks are
+ * area-downsampled to the target's patch resolution and averaged across the latent temporal
+ * spans; "Inputs you'll set": one static mask or one mask per prepared shot frame;
+ * "Common issues": any other mask length is an error).
+ *   mask              : device float array [F_in][Hp][Wp], row-major, values normally in [0,1]
+ *   F_in              : 1 (static mask) or shot_len (one mask per frame of the prepared shot)
+ *   shot_len          : frames of the prepared shot; must be 17n+5 (n >= 0)
+ *   frames_per_latent : tau, pixel frames per latent frame; latent frame f averages frames
+ *                       [f*tau, min((f+1)*tau, shot_len))
+ *   F_lat, Hq, Wq     : latent frames and patch grid of the target video
+ *   m_out             : device float array [F_lat][Hq][Wq] (written), i.e. the target
+ *                       tokens' m in packing order (frame-major, row-major patches)
+ * Cell (y, x) of a frame is the exact area average of the pixel image over
+ * [y*Hp/Hq, (y+1)*Hp/Hq) x [x*Wp/Wq, (x+1)*Wp/Wq).  A static mask is copied to every latent
+ * frame.  Errors: TARA_ERR_NULL, TARA_ERR_SHAPE (a size < 1, or latent frames beyond the
+ * shot), TARA_ERR_MASK_LENGTH, TARA_ERR_TOO_LARGE (F_lat > 65535 or Wq > 12288),
+ * TARA_ERR_ALIGN (4 bytes),
+ * TARA_ERR_CUDA; checked before launching.  Asynchronous on `stream`.                    */
+int tara_prepare_target_mask(const float* mask, int32_t F_in, int32_t Hp, int32_t Wp,
+                             int32_t shot_len, int32_t frames_per_latent, int32_t F_lat,
+                             int32_t Hq, int32_t Wq, float* m_out, void* stream);
 
 /* ---- the token-metadata packer (host) ------------------------------------------------- */
 /* One segment of the packed joint sequence, in packing order.  A segment is `frames` latent

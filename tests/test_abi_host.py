@@ -188,3 +188,26 @@ def test_packer_capacity_mismatch(lib):
                                   fb.ctypes.data, 11)
     assert rc == -8
     assert lib.tara_pack_token_meta(arr, 1, None, None, None, None, 10) == -1
+
+
+# ---------------------------------------------------------------------------------------
+# target-mask preparation: argument checks (fake pointers, rejected before any launch)
+# ---------------------------------------------------------------------------------------
+def _mask_call(lib, F_in=107, Hp=8, Wp=8, L=107, tau=4, F_lat=26, Hq=4, Wq=4, ptr=FAKE, out=FAKE):
+    return lib.tara_prepare_target_mask(ctypes.c_void_p(ptr), F_in, Hp, Wp, L, tau, F_lat, Hq,
+                                        Wq, ctypes.c_void_p(out), None)
+
+
+def test_mask_prep_argument_checks(lib):
+    assert _mask_call(lib, ptr=0) == -1
+    assert _mask_call(lib, out=0) == -1
+    assert _mask_call(lib, Hp=0) == -2
+    assert _mask_call(lib, tau=0) == -2
+    assert _mask_call(lib, F_in=360) == -12          # whole-clip mask into a 107-frame shot
+    assert _mask_call(lib, F_in=106) == -12
+    assert _mask_call(lib, L=108, F_in=108) == -12   # not a 17n+5 shot
+    assert _mask_call(lib, L=4, F_in=1) == -12
+    assert _mask_call(lib, F_lat=28) == -2           # latent frame 27 starts past the shot
+    assert _mask_call(lib, F_in=1, F_lat=70000) == -11
+    assert _mask_call(lib, Wq=20000) == -11
+    assert _mask_call(lib, ptr=FAKE + 2) == -6

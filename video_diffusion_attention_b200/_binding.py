@@ -22,11 +22,12 @@ STATUS = {
     0: "TARA_OK", -1: "TARA_ERR_NULL", -2: "TARA_ERR_SHAPE", -3: "TARA_ERR_DTYPE",
     -4: "TARA_ERR_HEAD_DIM", -5: "TARA_ERR_PARAM", -6: "TARA_ERR_ALIGN",
     -7: "TARA_ERR_SEGMENT", -8: "TARA_ERR_CAPACITY", -9: "TARA_ERR_CUDA",
-    -10: "TARA_ERR_DEVICE_TIMEOUT", -11: "TARA_ERR_TOO_LARGE",
+    -10: "TARA_ERR_DEVICE_TIMEOUT", -11: "TARA_ERR_TOO_LARGE", -12: "TARA_ERR_MASK_LENGTH",
 }
 EXPORTS = ("tara_default_params", "tara_status_string", "tara_attn_forward",
            "tara_device_status", "tara_packed_length", "tara_pack_token_meta",
-           "tara_set_kernel_events")
+           "tara_set_kernel_events", "tara_selftest_wait", "tara_attn_forward_noalloc",
+           "tara_prepare_target_mask")
 
 
 class TaraError(RuntimeError):
@@ -84,6 +85,11 @@ def load_library(path: Optional[str] = None):
     lib.tara_attn_forward_noalloc.argtypes = lib.tara_attn_forward.argtypes
     lib.tara_set_kernel_events.restype = ctypes.c_int
     lib.tara_set_kernel_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    lib.tara_prepare_target_mask.restype = ctypes.c_int
+    lib.tara_prepare_target_mask.argtypes = [ctypes.c_void_p] + [ctypes.c_int32] * 8 + [
+        ctypes.c_void_p, ctypes.c_void_p]
+    lib.tara_selftest_wait.restype = ctypes.c_int
+    lib.tara_selftest_wait.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
     lib.tara_device_status.restype = ctypes.c_int
     lib.tara_device_status.argtypes = [ctypes.c_void_p]
     lib.tara_packed_length.restype = ctypes.c_int64
@@ -259,6 +265,38 @@ def attn_forward_noalloc(q, k, v, meta: DeviceMeta, params: TaraParams, out, lse
     if rc != 0:
         raise TaraError(rc, "tara_attn_forward_noalloc")
     return out, lse
+
+
+def prepare_target_mask(mask, shot_len: int, frames_per_latent: int, F_lat: int, Hq: int,
+                        Wq: int, out=None, stream=None):
+    """Per-target-token mask weights [F_lat][Hq][Wq] from a device pixel mask [F_in][Hp][Wp]
+    (float32, contiguous), on the device (see include/tara_attn.h)."""
+    import torch
+    if mask.dim() != 3 or mask.dtype != torch.float32 or not mask.is_contiguous():
+        raise ValueError("mask must be a contiguous float32 [F][H][W] tensor")
+    F_in, Hp, Wp = (int(x) for x in mask.shape)
+    if out is None:
+        out = torch.empty((F_lat, Hq, Wq), dtype=torch.float32, device=mask.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(mask.device)
+    rc = load_library().tara_prepare_target_mask(
+        ctypes.c_void_p(mask.data_ptr()), F_in, Hp, Wp, int(shot_len), int(frames_per_latent),
+        int(F_lat), int(Hq), int(Wq), ctypes.c_void_p(out.data_ptr()),
+        ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise TaraError(rc, "tara_prepare_target_mask")
+    return out
+
+
+def selftest_wait(limit_us: int, arrive: bool, stream=None) -> None:
+    """Launch the bounded-wait self-test kernel (see include/tara_attn.h)."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    rc = load_library().tara_selftest_wait(int(limit_us), 1 if arrive else 0,
+                                          ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise TaraError(rc, "tara_selftest_wait")
 
 
 def device_status(stream=None) -> int:

@@ -12,6 +12,7 @@
 #include "attn_simt.cuh"
 #include "attn_pair.cuh"
 #include "attn_tc.cuh"
+#include "target_mask.cuh"
 #include "tile_summary.cuh"
 
 namespace tara {
@@ -149,6 +150,24 @@ int device_state(size_t bytes, DeviceState** out) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Self-test of the bounded-wait machinery: one warp waits on an mbarrier phase; with
+// arrive == 0 nothing ever arrives, so the wait must give up after limit_ns and set the
+// device status word exactly as an attention kernel does.
+__global__ void wait_selftest_kernel(int* status, uint64_t limit_ns, int arrive) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (arrive) mbar_arrive(&bar);
+    if (!mbar_wait(&bar, 0, &abort_flag, limit_ns)) atomicExch(status, 1);
+  }
+}
+
 template <bool kBF16, int D>
 int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
               const TcArgs& a, int B, int H, int ntiles, cudaStream_t stream, DeviceState* st) {
@@ -253,6 +272,7 @@ const char* tara_status_string(int s) {
     case TARA_ERR_CUDA: return "CUDA call failed";
     case TARA_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
     case TARA_ERR_TOO_LARGE: return "size too large";
+    case TARA_ERR_MASK_LENGTH: return "mask is neither one frame nor the prepared shot length";
     default: return "unknown status";
   }
 }
@@ -342,6 +362,36 @@ int tara_set_kernel_events(void* start, void* stop) {
   t_ev_start = static_cast<cudaEvent_t>(start);
   t_ev_stop = static_cast<cudaEvent_t>(stop);
   return TARA_OK;
+}
+
+int tara_prepare_target_mask(const float* mask, int32_t F_in, int32_t Hp, int32_t Wp,
+                             int32_t shot_len, int32_t frames_per_latent, int32_t F_lat,
+                             int32_t Hq, int32_t Wq, float* m_out, void* stream_) {
+  if (!mask || !m_out) return TARA_ERR_NULL;
+  if (F_in < 1 || Hp < 1 || Wp < 1 || frames_per_latent < 1 || F_lat < 1 || Hq < 1 || Wq < 1)
+    return TARA_ERR_SHAPE;
+  if (shot_len < 5 || (shot_len - 5) % 17 != 0) return TARA_ERR_MASK_LENGTH;
+  if (F_in != 1 && F_in != shot_len) return TARA_ERR_MASK_LENGTH;
+  if (F_in > 1 && (long long)(F_lat - 1) * frames_per_latent >= shot_len) return TARA_ERR_SHAPE;
+  if (F_lat > 65535 || Wq > 12288) return TARA_ERR_TOO_LARGE;   // Wq floats of shared memory
+  if ((reinterpret_cast<uintptr_t>(mask) & 3u) != 0 || (reinterpret_cast<uintptr_t>(m_out) & 3u) != 0)
+    return TARA_ERR_ALIGN;
+  dim3 grid((unsigned)Hq, (unsigned)(F_in > 1 ? F_lat : 1));
+  target_mask_kernel<<<grid, kMaskThreads, (size_t)Wq * sizeof(float),
+                       static_cast<cudaStream_t>(stream_)>>>(
+      mask, F_in, Hp, Wp, shot_len, frames_per_latent, F_lat, Hq, Wq, m_out);
+  return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
+}
+
+int tara_selftest_wait(int limit_us, int arrive, void* stream_) {
+  if (limit_us < 1 || limit_us > 10000000) return TARA_ERR_PARAM;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  int rc = device_state(0, &st);
+  if (rc != TARA_OK) return rc;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_)>>>(
+      st->status, (uint64_t)limit_us * 1000ull, arrive ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
 }
 
 int tara_device_status(void* stream_) {

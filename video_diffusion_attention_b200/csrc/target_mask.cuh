@@ -1,0 +1,108 @@
+// target_mask.cuh -- target-mask preparation on the device: a soft pixel mask (one frame, or
+// one per frame of the prepared shot) becomes one weight per target token, the value the
+// attention kernels read as m ("BFS H3 Reference Attention Binding (Experimental)": masks are
+// area-downsampled to the target's patch resolution and averaged across the latent temporal
+// spans).
+//
+// One CTA per (patch row y, latent frame f).  Its threads own pixel columns (thread t: columns
+// t, t + 256, ...), so every load of a pixel row is coalesced and each thread has many
+// independent loads in flight: per column they sum the pixels of the cell row's pixel rows
+// (weighted by each row's overlap with the cell row) over the latent frame's pixel frames.
+// The column sums are then added into the cells they overlap (shared-memory accumulators)
+// and normalised.  Overlaps are integers in units of 1/Hq pixel (rows) and 1/Wq pixel
+// (columns), so the area weights are exact.  HBM-bound: each pixel is read once (twice for a
+// pixel row straddling two cell rows).
+#pragma once
+
+#include <cstdint>
+
+namespace tara {
+
+constexpr int kMaskThreads = 256;
+constexpr int kMaskColsPerPass = 8;   // columns per thread per pass (register sums)
+
+__global__ void __launch_bounds__(kMaskThreads)
+target_mask_kernel(const float* __restrict__ mask, int F_in, int Hp, int Wp, int L, int tau,
+                   int F_lat, int Hq, int Wq, float* __restrict__ out) {
+  extern __shared__ float cell_acc[];   // [Wq]
+  const int y = blockIdx.x;
+  const int f = blockIdx.y;             // latent frame (0 when one static mask)
+  const int tid = threadIdx.x;
+
+  for (int x = tid; x < Wq; x += kMaskThreads) cell_acc[x] = 0.0f;
+  __syncthreads();
+
+  // pixel rows overlapping cell row y: [y*Hp, (y+1)*Hp) in units of 1/Hq pixel
+  const long long ylo = (long long)y * Hp, yhi = (long long)(y + 1) * Hp;
+  const int r0 = (int)(ylo / Hq);
+  const int r1 = (int)((yhi + Hq - 1) / Hq);          // exclusive
+  int t0 = 0, t1 = 1;
+  if (F_in > 1) {
+    t0 = f * tau;
+    t1 = min(t0 + tau, L);
+  }
+
+  // columns are handled in groups of 4 (one 16-byte load per pixel row) when every row starts
+  // on a 16-byte boundary, else one at a time
+  const bool vec4 = (Wp % 4 == 0) && ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0);
+  // a pass covers 2048 columns: 8 register sums per thread (2 x 4 columns, or 8 x 1)
+  constexpr int kSlots = kMaskColsPerPass;
+  for (int base = 0; base < Wp; base += kMaskThreads * kSlots) {
+    float colsum[kSlots];
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) colsum[k] = 0.0f;
+    for (int t = t0; t < t1; ++t) {
+#pragma unroll 2
+      for (int r = r0; r < r1; ++r) {
+        const long long rlo = (long long)r * Hq;
+        const float wy = (float)(min(yhi, rlo + Hq) - max(ylo, rlo));
+        const float* row = mask + ((long long)t * Hp + r) * Wp;
+        if (vec4) {
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int c = base + (k * kMaskThreads + tid) * 4;
+            if (c < Wp) {
+              const float4 v = __ldg(reinterpret_cast<const float4*>(row + c));
+              colsum[4 * k + 0] = fmaf(wy, v.x, colsum[4 * k + 0]);
+              colsum[4 * k + 1] = fmaf(wy, v.y, colsum[4 * k + 1]);
+              colsum[4 * k + 2] = fmaf(wy, v.z, colsum[4 * k + 2]);
+              colsum[4 * k + 3] = fmaf(wy, v.w, colsum[4 * k + 3]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < kSlots; ++k) {
+            const int c = base + k * kMaskThreads + tid;
+            if (c < Wp) colsum[k] = fmaf(wy, __ldg(row + c), colsum[k]);
+          }
+        }
+      }
+    }
+    // add each column sum into the cells the column overlaps, weighted by the overlap
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) {
+      const int c = vec4 ? base + ((k >> 2) * kMaskThreads + tid) * 4 + (k & 3)
+                         : base + k * kMaskThreads + tid;
+      if (c >= Wp) continue;
+      const long long clo = (long long)c * Wq, chi = clo + Wq;
+      for (int x = (int)(clo / Wp); x < Wq && (long long)x * Wp < chi; ++x) {
+        const long long xlo = (long long)x * Wp;
+        const float wx = (float)(min(xlo + Wp, chi) - max(xlo, clo));
+        atomicAdd(&cell_acc[x], wx * colsum[k]);
+      }
+    }
+  }
+  __syncthreads();
+
+  const float norm = 1.0f / ((float)Hp * (float)Wp * (float)(t1 - t0));
+  for (int x = tid; x < Wq; x += kMaskThreads) {
+    const float v = cell_acc[x] * norm;
+    if (F_in > 1) {
+      out[((long long)f * Hq + y) * Wq + x] = v;
+    } else {
+      for (int ff = 0; ff < F_lat; ++ff) out[((long long)ff * Hq + y) * Wq + x] = v;
+    }
+  }
+}
+
+}  // namespace tara

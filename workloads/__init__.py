@@ -107,6 +107,25 @@ def ellipse_mask(seed: int, rows: int = 40, cols: int = 50) -> np.ndarray:
     return (1.0 / (1.0 + np.exp((r - 1.0) / 0.1))).astype(np.float32).reshape(-1)
 
 
+def pixel_ellipse_mask(seed: int, frames: int, height: int, width: int) -> np.ndarray:
+    """Soft elliptic pixel mask [frames][height][width] (float32) whose centre drifts linearly
+    across the frames (a tracked subject); same edge profile as `ellipse_mask`."""
+    g = np.random.Generator(np.random.PCG64(seed))
+    cy0, cy1 = g.uniform(height * 0.3, height * 0.7, size=2)
+    cx0, cx1 = g.uniform(width * 0.3, width * 0.7, size=2)
+    ay = g.uniform(0.2, 0.4) * height
+    ax = g.uniform(0.2, 0.4) * width
+    y = np.arange(height, dtype=np.float64)[:, None] + 0.5
+    x = np.arange(width, dtype=np.float64)[None, :] + 0.5
+    out = np.empty((frames, height, width), dtype=np.float32)
+    for f in range(frames):
+        a = f / max(1, frames - 1)
+        cy, cx = cy0 + a * (cy1 - cy0), cx0 + a * (cx1 - cx0)
+        r = np.sqrt(((y - cy) / ay) ** 2 + ((x - cx) / ax) ** 2)
+        out[f] = (1.0 / (1.0 + np.exp((r - 1.0) / 0.1))).astype(np.float32)
+    return out
+
+
 def uniform_mask(seed: int, n: int) -> np.ndarray:
     g = np.random.Generator(np.random.PCG64(seed))
     return g.uniform(0.0, 1.0, size=n).astype(np.float32)
