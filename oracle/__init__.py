@@ -54,25 +54,29 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def _bind(lib):
+    """Declare the C signatures on a loaded oracle library (the built one, or a test's copy)."""
+    lib.oracle_attention_rows.restype = ctypes.c_int
+    lib.oracle_attention_rows.argtypes = (
+        [ctypes.c_void_p] * 3 + [ctypes.c_int] + [ctypes.c_int64] * 4 +
+        [ctypes.c_void_p] * 4 + [ctypes.c_int64] + [ctypes.c_double] * 4 +
+        [ctypes.c_void_p, ctypes.c_double, ctypes.c_void_p, ctypes.c_int64,
+         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int])
+    lib.oracle_penalty.restype = ctypes.c_double
+    lib.oracle_penalty.argtypes = [ctypes.c_double] * 5
+    lib.oracle_max_threads.restype = ctypes.c_int
+    lib.oracle_logit_row.restype = ctypes.c_int
+    lib.oracle_logit_row.argtypes = (
+        [ctypes.c_void_p] * 2 + [ctypes.c_int] + [ctypes.c_int64] * 4 +
+        [ctypes.c_void_p] * 4 + [ctypes.c_int64] + [ctypes.c_double] * 4 +
+        [ctypes.c_void_p, ctypes.c_double] + [ctypes.c_int64] * 3 + [ctypes.c_void_p])
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        lib.oracle_attention_rows.restype = ctypes.c_int
-        lib.oracle_attention_rows.argtypes = (
-            [ctypes.c_void_p] * 3 + [ctypes.c_int] + [ctypes.c_int64] * 4 +
-            [ctypes.c_void_p] * 4 + [ctypes.c_int64] + [ctypes.c_double] * 4 +
-            [ctypes.c_void_p, ctypes.c_double, ctypes.c_void_p, ctypes.c_int64,
-             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int])
-        lib.oracle_penalty.restype = ctypes.c_double
-        lib.oracle_penalty.argtypes = [ctypes.c_double] * 5
-        lib.oracle_max_threads.restype = ctypes.c_int
-        lib.oracle_logit_row.restype = ctypes.c_int
-        lib.oracle_logit_row.argtypes = (
-            [ctypes.c_void_p] * 2 + [ctypes.c_int] + [ctypes.c_int64] * 4 +
-            [ctypes.c_void_p] * 4 + [ctypes.c_int64] + [ctypes.c_double] * 4 +
-            [ctypes.c_void_p, ctypes.c_double] + [ctypes.c_int64] * 3 + [ctypes.c_void_p])
-        _lib = lib
+        _lib = _bind(ctypes.CDLL(build()))
     return _lib
 
 
