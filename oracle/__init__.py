@@ -12,6 +12,8 @@ Sources, by page and section:
     only; defaults window 0.20 s, falloff 0.25 s, strength 2.0, cap 6.0.
   - "BFS H3 Reference Attention Binding (Experimental)", "The exact rule": a target-video
     query with mask weight m and a key of Picture i gain m*log(gain_i) on the logit.
+  - "BFS H3 Reference Attention Binding", "Common issues": chained bindings (one per subject)
+    combine their log gains: binding k adds m_k * log(gain_k,i) for its own mask m_k.
   - "TARA: ...", "Three backends": the output is attention with its log-sum-exp.
 
 Readings taken where the pages are silent (each also listed in the design notes):
@@ -61,7 +63,8 @@ def _bind(lib):
         [ctypes.c_void_p] * 3 + [ctypes.c_int] + [ctypes.c_int64] * 4 +
         [ctypes.c_void_p] * 4 + [ctypes.c_int64] + [ctypes.c_double] * 4 +
         [ctypes.c_void_p, ctypes.c_double, ctypes.c_void_p, ctypes.c_int64,
-         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int])
+         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+         ctypes.c_void_p, ctypes.c_int64])
     lib.oracle_penalty.restype = ctypes.c_double
     lib.oracle_penalty.argtypes = [ctypes.c_double] * 5
     lib.oracle_max_threads.restype = ctypes.c_int
@@ -69,7 +72,8 @@ def _bind(lib):
     lib.oracle_logit_row.argtypes = (
         [ctypes.c_void_p] * 2 + [ctypes.c_int] + [ctypes.c_int64] * 4 +
         [ctypes.c_void_p] * 4 + [ctypes.c_int64] + [ctypes.c_double] * 4 +
-        [ctypes.c_void_p, ctypes.c_double] + [ctypes.c_int64] * 3 + [ctypes.c_void_p])
+        [ctypes.c_void_p, ctypes.c_double] + [ctypes.c_int64] * 3 + [ctypes.c_void_p] +
+        [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64])
     return lib
 
 
@@ -130,6 +134,18 @@ def _as_float32(x) -> float:
     return float(np.float32(x))
 
 
+def _extra(meta: Dict, params, cv):
+    """(n, gains [n*9] float64, masks [n][m_len] float32, m_len) of the extra bindings."""
+    gains = list(getattr(params, "extra_gain", ()) or ())
+    n = len(gains)
+    if n == 0:
+        return 0, None, None, 0
+    g = np.ascontiguousarray([[cv(x) for x in row] for row in gains], dtype=np.float64)
+    assert g.shape == (n, 9)
+    mm = np.ascontiguousarray(meta["m_extra"], dtype=np.float32).reshape(n, -1)
+    return n, g, mm, mm.shape[1]
+
+
 def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, dtype: str, meta: Dict,
                    params, rows: np.ndarray, meta_batch_stride: int = 0,
                    n_threads: int = 0, params_as_float32: bool = True):
@@ -159,12 +175,14 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, dtype: str, meta
     scale = cv(params.softmax_scale) if params.softmax_scale else 0.0
     O = np.empty((n, D), dtype=np.float64)
     L = np.empty((n,), dtype=np.float64)
+    ne, eg, em, mlen = _extra(meta, params, cv)
     rc = lib.oracle_attention_rows(
         q.ctypes.data, k.ctypes.data, v.ctypes.data, _DTYPE_CODE[dtype], B, H, N, D,
         seg.ctypes.data, ts.ctypes.data, pic.ctypes.data, m.ctypes.data, int(meta_batch_stride),
         cv(params.window), cv(params.falloff), cv(params.strength), cv(params.cap),
         gain.ctypes.data, scale, rows.ctypes.data, n, O.ctypes.data, L.ctypes.data,
-        int(n_threads))
+        int(n_threads), ne, None if eg is None else eg.ctypes.data,
+        None if em is None else em.ctypes.data, mlen)
     if rc != 0:
         raise RuntimeError("oracle_attention_rows failed")
     return O, L
@@ -183,11 +201,13 @@ def logit_row(q, k, dtype: str, meta: Dict, params, b: int, h: int, i: int,
     m = np.ascontiguousarray(meta["m"], dtype=np.float32)
     out = np.empty((N,), dtype=np.float64)
     scale = cv(params.softmax_scale) if params.softmax_scale else 0.0
+    ne, eg, em, mlen = _extra(meta, params, cv)
     rc = lib.oracle_logit_row(q.ctypes.data, k.ctypes.data, _DTYPE_CODE[dtype], B, H, N, D,
                               seg.ctypes.data, ts.ctypes.data, pic.ctypes.data, m.ctypes.data,
                               int(meta_batch_stride), cv(params.window), cv(params.falloff),
                               cv(params.strength), cv(params.cap), gain.ctypes.data, scale,
-                              b, h, i, out.ctypes.data)
+                              b, h, i, out.ctypes.data, ne, None if eg is None else eg.ctypes.data,
+                              None if em is None else em.ctypes.data, mlen)
     if rc != 0:
         raise RuntimeError("oracle_logit_row failed")
     return out

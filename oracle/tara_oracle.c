@@ -17,6 +17,8 @@
  *   if token i is TARGET and token j is PICTURE p ("BFS H3 Reference Attention Binding
  *                                                (Experimental)", "The exact rule")
  *     s_j = s_j + m_i * ln(gain_p)
+ *           + sum over extra bindings k of m_k,i * ln(gain_k,p)   ("Common issues":
+ *                                                chained bindings combine their log gains)
  *   M = max_j s_j,  l = sum_j exp(s_j - M),  LSE_i = M + ln l,
  *   O_i = sum_j exp(s_j - M) * V[b,h,j,:] / l
  *
@@ -64,10 +66,22 @@ double oracle_penalty(double dt, double window, double falloff, double strength,
   return p < cap ? p : cap;
 }
 
+/* Extra reference bindings beyond the first ("BFS H3 Reference Attention Binding
+ * (Experimental)", "Common issues": two subjects are two chained binding nodes, and
+ * overlapping masks combine their log gains).  Binding k has its own 9 gains and its own mask
+ * weight per token (m_extra + k * m_len, offset to the branch like m). */
+typedef struct {
+  int n;                  /* extra bindings, 0..3 */
+  const double* gains;    /* n x 9 */
+  const float* m;         /* n arrays of m_len floats */
+  int64_t m_len;
+} oracle_bindings;
+
 /* Bias of the edge (query token i, key token j); meta arrays already offset to the branch. */
 double oracle_bias(int64_t i, int64_t j, const uint8_t* seg, const float* time_s,
                    const uint8_t* pic, const float* m, double window, double falloff,
-                   double strength, double cap, const double* gain9) {
+                   double strength, double cap, const double* gain9,
+                   const oracle_bindings* extra, int64_t mo) {
   if (seg[i] != ROLE_TARGET) return 0.0;
   if (seg[j] == ROLE_GUIDE) {
     double dt = fabs((double)time_s[i] - (double)time_s[j]);
@@ -76,7 +90,10 @@ double oracle_bias(int64_t i, int64_t j, const uint8_t* seg, const float* time_s
   if (seg[j] == ROLE_PICTURE) {
     int p = pic[j];
     if (p < 1 || p > 9) return 0.0;
-    return (double)m[i] * log(gain9[p - 1]);
+    double b = (double)m[i] * log(gain9[p - 1]);
+    for (int k = 0; extra && k < extra->n; ++k)
+      b += (double)extra->m[k * extra->m_len + mo + i] * log(extra->gains[9 * k + p - 1]);
+    return b;
   }
   return 0.0;
 }
@@ -94,11 +111,15 @@ int oracle_attention_rows(const void* Q, const void* K, const void* V, int dtype
                           double window, double falloff, double strength, double cap,
                           const double* gain9, double scale,
                           const int64_t* rows, int64_t n_rows,
-                          double* O_out, double* LSE_out, int n_threads) {
+                          double* O_out, double* LSE_out, int n_threads,
+                          int n_extra, const double* extra_gains, const float* extra_m,
+                          int64_t m_len) {
   if (!Q || !K || !V || !seg || !time_s || !pic || !m || !gain9 || !rows || !O_out || !LSE_out)
     return -1;
   if (B < 1 || H < 1 || N < 1 || D < 1 || n_rows < 0) return -1;
+  if (n_extra < 0 || n_extra > 3 || (n_extra > 0 && (!extra_gains || !extra_m))) return -1;
   if (scale == 0.0) scale = 1.0 / sqrt((double)D);
+  const oracle_bindings extra = {n_extra, extra_gains, extra_m, m_len};
   int failed = 0;
 #ifdef _OPENMP
   if (n_threads > 0) omp_set_num_threads(n_threads);
@@ -133,7 +154,7 @@ int oracle_attention_rows(const void* Q, const void* K, const void* V, int dtype
           double dot = 0.0;
           for (int64_t k = 0; k < D; ++k) dot += q[k] * widen(K, dtype, head + j * D + k);
           double sj = dot * scale + oracle_bias(i, j, seg + mo, time_s + mo, pic + mo, m + mo,
-                                                window, falloff, strength, cap, gain9);
+                                                window, falloff, strength, cap, gain9, &extra, mo);
           s[j] = sj;
           if (sj > M) M = sj;
         }
@@ -162,8 +183,11 @@ int oracle_logit_row(const void* Q, const void* K, int dtype, int64_t B, int64_t
                      int64_t D, const uint8_t* seg, const float* time_s, const uint8_t* pic,
                      const float* m, int64_t meta_batch_stride, double window, double falloff,
                      double strength, double cap, const double* gain9, double scale,
-                     int64_t b, int64_t h, int64_t i, double* out) {
+                     int64_t b, int64_t h, int64_t i, double* out, int n_extra,
+                     const double* extra_gains, const float* extra_m, int64_t m_len) {
   if (!Q || !K || !seg || !time_s || !pic || !m || !gain9 || !out) return -1;
+  if (n_extra < 0 || n_extra > 3 || (n_extra > 0 && (!extra_gains || !extra_m))) return -1;
+  const oracle_bindings extra = {n_extra, extra_gains, extra_m, m_len};
   if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= N || D < 1) return -1;
   if (scale == 0.0) scale = 1.0 / sqrt((double)D);
   int64_t head = (b * H + h) * N * D;
@@ -173,7 +197,7 @@ int oracle_logit_row(const void* Q, const void* K, int dtype, int64_t B, int64_t
     for (int64_t k = 0; k < D; ++k)
       dot += widen(Q, dtype, head + i * D + k) * widen(K, dtype, head + j * D + k);
     out[j] = dot * scale + oracle_bias(i, j, seg + mo, time_s + mo, pic + mo, m + mo, window,
-                                       falloff, strength, cap, gain9);
+                                       falloff, strength, cap, gain9, &extra, mo);
   }
   return 0;
 }

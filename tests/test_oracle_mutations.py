@@ -25,10 +25,15 @@ MUTANTS = {
     "window dropped": ("double x = dt - window;", "double x = dt;"),
     "falloff multiplies": ("x = x / falloff;", "x = x * falloff;"),
     "cap ignored": ("return p < cap ? p : cap;", "return p;"),
-    "mask weight dropped": ("return (double)m[i] * log(gain9[p - 1]);",
-                            "return log(gain9[p - 1]);"),
-    "picture index off by one": ("return (double)m[i] * log(gain9[p - 1]);",
-                                 "return (double)m[i] * log(gain9[p % 9]);"),
+    "mask weight dropped": ("double b = (double)m[i] * log(gain9[p - 1]);",
+                            "double b = log(gain9[p - 1]);"),
+    "picture index off by one": ("double b = (double)m[i] * log(gain9[p - 1]);",
+                                 "double b = (double)m[i] * log(gain9[p % 9]);"),
+    "extra binding reuses the first gains": ("* log(extra->gains[9 * k + p - 1]);",
+                                             "* log(gain9[p - 1]);"),
+    "extra binding ignores its mask": ("b += (double)extra->m[k * extra->m_len + mo + i] *",
+                                       "b += 1.0 *"),
+    "extra bindings replace instead of add": ("b += (double)extra->m[", "b = (double)extra->m["),
     "values used as keys": ("dot += q[k] * widen(K, dtype, head + j * D + k);",
                             "dot += q[k] * widen(V, dtype, head + j * D + k);"),
     "lse without max": ("LSE_out[r] = M + log(l);", "LSE_out[r] = log(l);"),

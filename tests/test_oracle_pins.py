@@ -182,7 +182,7 @@ def _edge_weights(q, k, meta, p):
     qn = np.zeros((B, H, N, N)); qn[..., :D] = q
     kn = np.zeros((B, H, N, N)); kn[..., :D] = k
     p2 = W.Params(p.window, p.falloff, p.strength, p.cap, p.gain,
-                  softmax_scale=1.0 / math.sqrt(D))
+                  softmax_scale=1.0 / math.sqrt(D), extra_gain=p.extra_gain)
     O, L = run_all(qn, kn, v, meta, p2)
     return O * np.exp(L)[..., None]
 
@@ -399,3 +399,68 @@ def test_packer_clock_and_roles(golden_rule):
     assert np.all(rg["m"] == 1.0)
     gt = rg["time_s"][rg["seg"] == W.GUIDE].reshape(26, 461)
     np.testing.assert_array_equal(gt[:, 0], (np.arange(26) * 4 / fps + 1 / fps).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------------------
+# chained bindings ("Common issues": two subjects are two chained binding nodes; overlapping
+# masks combine their log gains)
+# ---------------------------------------------------------------------------------------
+def _two_bindings(seed, m2_fn):
+    q, k, v, meta, _ = tiny_case(seed=seed)
+    N = len(meta["seg"])
+    rng = np.random.Generator(np.random.PCG64(seed + 50))
+    m2 = np.ones(N, dtype=np.float32)
+    tgt = meta["seg"] == W.TARGET
+    m2[tgt] = m2_fn(rng, int(tgt.sum()))
+    meta = dict(meta, m_extra=m2[None, :])
+    g1 = (1.25, 0.75) + (1.0,) * 7            # binding 0: Picture 1 chosen
+    g2 = (0.9, 1.6) + (0.9,) * 7              # binding 1: Picture 2 chosen
+    p = W.Params(gain=g1, extra_gain=(g2,))
+    return q, k, meta, p, g1, g2, m2
+
+
+def test_overlapping_bindings_multiply_gain_powers():
+    q, k, meta, p, g1, g2, m2 = _two_bindings(20, lambda rng, n: rng.uniform(0, 1, n))
+    neutral = W.Params(p.window, p.falloff, p.strength, p.cap, (1.0,) * 9)
+    ratio = _edge_weights(q, k, meta, p) / _edge_weights(q, k, {kk: vv for kk, vv in meta.items() if kk != "m_extra"}, neutral)
+    seg, pic, m = meta["seg"], meta["pic"], meta["m"].astype(np.float64)
+    f32 = lambda g: np.array([float(np.float32(x)) for x in g])
+    a, b = f32(g1), f32(g2)
+    N = len(seg)
+    for i in range(N):
+        for j in range(N):
+            if seg[i] == W.TARGET and seg[j] == W.PICTURE:
+                expect = a[pic[j] - 1] ** m[i] * b[pic[j] - 1] ** float(m2[i])
+            else:
+                expect = 1.0
+            assert ratio[0, 0, i, j] == pytest.approx(expect, rel=1e-12, abs=0), (i, j)
+
+
+def test_extra_binding_with_zero_mask_changes_nothing():
+    q, k, meta, p, g1, g2, m2 = _two_bindings(21, lambda rng, n: np.zeros(n))
+    v = np.random.Generator(np.random.PCG64(9)).standard_normal(q.shape)
+    O1, L1 = run_all(q, k, v, meta, p)
+    single = W.Params(gain=g1)
+    O0, L0 = run_all(q, k, v, {kk: vv for kk, vv in meta.items() if kk != "m_extra"}, single)
+    np.testing.assert_array_equal(O1, O0)
+    np.testing.assert_array_equal(L1, L0)
+
+
+def test_disjoint_bindings_act_on_their_own_rows():
+    # binding 0 masks the first half of the target rows, binding 1 the second half
+    q, k, meta, p, g1, g2, m2 = _two_bindings(22, lambda rng, n: (np.arange(n) >= n // 2).astype(np.float32))
+    tgt = np.where(meta["seg"] == W.TARGET)[0]
+    m = meta["m"].copy()
+    m[tgt] = (np.arange(len(tgt)) < len(tgt) // 2).astype(np.float32)
+    meta = dict(meta, m=m)
+    v = np.random.Generator(np.random.PCG64(10)).standard_normal(q.shape)
+    O, L = run_all(q, k, v, meta, p)
+    no_extra = {kk: vv for kk, vv in meta.items() if kk != "m_extra"}
+    Oa, La = run_all(q, k, v, no_extra, W.Params(gain=g1))
+    m_b = m.copy()
+    m_b[tgt] = m2[tgt]
+    Ob, Lb = run_all(q, k, v, dict(no_extra, m=m_b), W.Params(gain=g2))
+    first, second = tgt[: len(tgt) // 2], tgt[len(tgt) // 2:]
+    np.testing.assert_allclose(O[:, :, first], Oa[:, :, first], atol=1e-13, rtol=0)
+    np.testing.assert_allclose(O[:, :, second], Ob[:, :, second], atol=1e-13, rtol=0)
+    np.testing.assert_allclose(L[:, :, second], Lb[:, :, second], atol=1e-13, rtol=0)

@@ -56,6 +56,7 @@ class Params:
     cap: float = 6.0
     gain: tuple = (1.0,) * 9
     softmax_scale: float = 0.0          # 0: 1/sqrt(D)
+    extra_gain: tuple = ()              # gains (9 each) of chained bindings beyond the first
 
 
 @dataclasses.dataclass
