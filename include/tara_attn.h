@@ -14,7 +14,7 @@
  *               selected motion (GUIDE) video
  *               ("TARA: Native Temporal Alignment for MiniMax H3 References",
  *                section "The temporal rule");
- *           = m_i * ln(gain[pic_j])
+ *           = m_i * ln(gain[pic_j])  (+ the same term of every extra chained binding)
  *               if token i is a TARGET token with mask weight m_i and token j belongs to
  *               native Picture pic_j
  *               ("BFS H3 Reference Attention Binding (Experimental)", section "The exact rule");
@@ -104,6 +104,11 @@ typedef struct {
   const float*   m;
   int32_t        N;
   int64_t        batch_stride;
+  /* Masks of the extra (chained) bindings, see tara_params.n_extra_bindings: binding k's
+   * weight of token i (set b) is extra_m[k * extra_m_stride + b * batch_stride + i].  Device
+   * pointer; may be NULL when there are no extra bindings.                                */
+  const float*   extra_m;
+  int64_t        extra_m_stride;
 } tara_token_meta;
 
 /* Rule parameters.  Defaults ("TARA: ...", "The temporal rule"): window 0.20 s,
@@ -112,13 +117,23 @@ typedef struct {
  * chosen Picture, other_reference_strength for the others, 1 = neutral).
  * Domain: falloff > 0; window, strength, cap >= 0; gain > 0; all finite.
  * softmax_scale: 0 selects 1/sqrt(D); otherwise a finite positive value used as is.        */
+#define TARA_MAX_EXTRA_BINDINGS 3
+
 typedef struct {
   float window, falloff, strength, cap;
   float gain[9];
   float softmax_scale;
+  /* Chained bindings ("BFS H3 Reference Attention Binding", "Common issues": two subjects are
+   * two chained binding nodes, and overlapping masks combine their log gains).  gain[] with
+   * token_meta.m is the first binding; extra binding k (k < n_extra_bindings <= 3) has its own
+   * gains extra_gain[k][i-1] and its own mask (token_meta.extra_m).  A target query i and a
+   * key of Picture p then get m_i ln(gain[p-1]) + sum_k m_k,i ln(extra_gain[k][p-1]).        */
+  int32_t n_extra_bindings;
+  float extra_gain[TARA_MAX_EXTRA_BINDINGS][9];
 } tara_params;
 
-/* Fill *p with the defaults above (all gains 1, softmax_scale 0).  NULL is ignored. */
+/* Fill *p with the defaults above (all gains 1, softmax_scale 0, no extra bindings).  NULL
+ * is ignored. */
 void tara_default_params(tara_params* p);
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -135,6 +150,8 @@ const char* tara_status_string(int status);
  *   LSE     : device float array [B][H][N] (written).
  *   stream  : CUDA stream (cudaStream_t), 0 for the legacy default stream.
  * Every O row and LSE entry is written; no other memory of the caller is touched.
+ * Extra bindings: 0..3; their gains follow the same domain; extra_m must be non-NULL and
+ * 4-byte aligned when there are any, and extra_m_stride at least the length of one m array.
  * Errors: TARA_ERR_NULL, _SHAPE, _DTYPE, _HEAD_DIM, _PARAM, _ALIGN, _TOO_LARGE (checked
  * before any launch), TARA_ERR_CUDA (workspace allocation or launch failure).             */
 int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,

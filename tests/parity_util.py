@@ -16,25 +16,33 @@ TOL = {
 }
 
 
-def run_gpu(w: W.Workload, q, k, v, per_branch_meta: bool = False):
-    """O, LSE from the CUDA path (through the C ABI) for workload w on cuda tensors q, k, v."""
+def _with_extra(meta: dict, m_extra, copies: int = 1) -> dict:
+    if m_extra is not None:
+        meta["m_extra"] = np.concatenate([np.asarray(m_extra, np.float32)] * copies, axis=1)
+    return meta
+
+
+def run_gpu(w: W.Workload, q, k, v, per_branch_meta: bool = False, m_extra=None):
+    """O, LSE from the CUDA path (through the C ABI) for workload w on cuda tensors q, k, v.
+
+    m_extra: [n][N] masks of the chained bindings named by w.params.extra_gain (or None)."""
     import video_diffusion_attention_b200 as T
     meta = T.pack_token_meta(w.segments)
     if per_branch_meta:
         N = len(meta["seg"])
         stacked = {key: np.concatenate([val] * w.B) for key, val in meta.items()}
-        dmeta = T.DeviceMeta(stacked, q.device, batch_stride=N, N=N)
+        dmeta = T.DeviceMeta(_with_extra(stacked, m_extra, w.B), q.device, batch_stride=N, N=N)
     else:
-        dmeta = T.DeviceMeta(meta, q.device)
+        dmeta = T.DeviceMeta(_with_extra(meta, m_extra), q.device)
     O, L = T.attn_forward(q, k, v, dmeta, T.params_from(w.params))
     torch.cuda.synchronize()
     assert T.device_status() == 0
     return O, L
 
 
-def run_oracle(w: W.Workload, q, k, v, rows: np.ndarray):
+def run_oracle(w: W.Workload, q, k, v, rows: np.ndarray, m_extra=None):
     """O, LSE (fp64) of the oracle on host copies of the same tensors, for rows (b, h, i)."""
-    meta = oracle.pack_token_meta(w.segments)
+    meta = _with_extra(oracle.pack_token_meta(w.segments), m_extra)
     raw = [oracle.torch_to_numpy_raw(t) for t in (q, k, v)]
     return oracle.attention_rows(raw[0][0], raw[1][0], raw[2][0], raw[0][1], meta, w.params,
                                  rows)

@@ -68,11 +68,12 @@ def _t(ptr=FAKE, dtype=B.TARA_BF16, shape=(1, 2, 300, 128)):
     return t
 
 
-def _meta(N=300, stride=0, ptr=FAKE):
+def _meta(N=300, stride=0, ptr=FAKE, extra=None, extra_stride=0):
     m = B.TaraTokenMeta()
     m.seg = m.pic = ptr
     m.time_s = m.m = ptr
     m.N, m.batch_stride = N, stride
+    m.extra_m, m.extra_m_stride = extra, extra_stride
     return m
 
 
@@ -133,6 +134,47 @@ def test_rejects_misalignment(lib):
 ])
 def test_rejects_parameters(lib, kw):
     assert _call(lib, p=B.make_params(**kw)) == -5
+
+
+def test_default_params_have_no_extra_bindings(lib):
+    p = B.default_params()
+    assert p.n_extra_bindings == 0
+    assert all(p.extra_gain[k][i] == 1.0 for k in range(B.MAX_EXTRA_BINDINGS) for i in range(9))
+
+
+def _extra_params(n, bad=None):
+    p = B.make_params()
+    p.n_extra_bindings = n
+    for k in range(B.MAX_EXTRA_BINDINGS):
+        for i in range(9):
+            p.extra_gain[k][i] = 1.0
+    if bad is not None:
+        p.extra_gain[min(n, B.MAX_EXTRA_BINDINGS) - 1][4] = bad
+    return p
+
+
+def test_extra_binding_checks(lib):
+    ok_meta = _meta(extra=FAKE, extra_stride=300)
+    for n in (-1, 4, 1000):
+        assert _call(lib, meta=ok_meta, p=_extra_params(n)) == -5
+    for bad in (0.0, -2.0, float("inf"), float("nan")):
+        assert _call(lib, meta=ok_meta, p=_extra_params(2, bad)) == -5
+    assert _call(lib, meta=_meta(extra=None, extra_stride=300), p=_extra_params(1)) == -1
+    assert _call(lib, meta=_meta(extra=FAKE, extra_stride=299), p=_extra_params(1)) == -2
+    # batch-strided metadata: each mask spans (B-1)*stride + N entries
+    s2 = (2, 2, 300, 128)
+    t2 = dict(Q=_t(shape=s2), K=_t(shape=s2), V=_t(shape=s2), O=_t(shape=s2))
+    assert _call(lib, meta=_meta(stride=320, extra=FAKE, extra_stride=619),
+                 p=_extra_params(1), **t2) == -2
+    assert _call(lib, meta=_meta(extra=FAKE + 2, extra_stride=300), p=_extra_params(1)) == -6
+    # gains of unused binding slots are not read
+    p = _extra_params(1)
+    p.extra_gain[2][0] = -1.0
+    assert _call(lib, meta=_meta(extra=FAKE, extra_stride=300, ptr=0), p=p) == -1
+    with pytest.raises(ValueError):
+        B.make_params(extra_gain=((1.0,) * 9,) * 4)
+    with pytest.raises(ValueError):
+        B.make_params(extra_gain=((1.0,) * 8,))
 
 
 # ---------------------------------------------------------------------------------------

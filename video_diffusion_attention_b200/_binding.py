@@ -41,16 +41,22 @@ class TaraTensor(ctypes.Structure):
                 ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("D", ctypes.c_int32)]
 
 
+MAX_EXTRA_BINDINGS = 3   # TARA_MAX_EXTRA_BINDINGS
+
+
 class TaraTokenMeta(ctypes.Structure):
     _fields_ = [("seg", ctypes.c_void_p), ("time_s", ctypes.c_void_p),
                 ("pic", ctypes.c_void_p), ("m", ctypes.c_void_p), ("N", ctypes.c_int32),
-                ("batch_stride", ctypes.c_int64)]
+                ("batch_stride", ctypes.c_int64), ("extra_m", ctypes.c_void_p),
+                ("extra_m_stride", ctypes.c_int64)]
 
 
 class TaraParams(ctypes.Structure):
     _fields_ = [("window", ctypes.c_float), ("falloff", ctypes.c_float),
                 ("strength", ctypes.c_float), ("cap", ctypes.c_float),
-                ("gain", ctypes.c_float * 9), ("softmax_scale", ctypes.c_float)]
+                ("gain", ctypes.c_float * 9), ("softmax_scale", ctypes.c_float),
+                ("n_extra_bindings", ctypes.c_int32),
+                ("extra_gain", (ctypes.c_float * 9) * MAX_EXTRA_BINDINGS)]
 
 
 class TaraSegment(ctypes.Structure):
@@ -106,7 +112,8 @@ def load_library(path: Optional[str] = None):
 # parameters and packing
 # ---------------------------------------------------------------------------------------
 def make_params(window=0.20, falloff=0.25, strength=2.0, cap=6.0, gain=(1.0,) * 9,
-                softmax_scale=0.0) -> TaraParams:
+                softmax_scale=0.0, extra_gain=()) -> TaraParams:
+    """TaraParams; extra_gain lists the 9 gains of each chained binding beyond the first."""
     p = TaraParams()
     p.window, p.falloff, p.strength, p.cap = window, falloff, strength, cap
     g = list(gain)
@@ -115,13 +122,21 @@ def make_params(window=0.20, falloff=0.25, strength=2.0, cap=6.0, gain=(1.0,) * 
     for i in range(9):
         p.gain[i] = g[i]
     p.softmax_scale = softmax_scale
+    extra = [list(row) for row in extra_gain]
+    if len(extra) > MAX_EXTRA_BINDINGS or any(len(row) != 9 for row in extra):
+        raise ValueError("extra_gain: at most %d bindings of 9 gains" % MAX_EXTRA_BINDINGS)
+    p.n_extra_bindings = len(extra)
+    for k in range(MAX_EXTRA_BINDINGS):
+        for i in range(9):
+            p.extra_gain[k][i] = extra[k][i] if k < len(extra) else 1.0
     return p
 
 
 def params_from(obj) -> TaraParams:
-    """TaraParams from any object with window, falloff, strength, cap, gain, softmax_scale."""
+    """TaraParams from any object with window, falloff, strength, cap, gain, softmax_scale
+    (and optionally extra_gain)."""
     return make_params(obj.window, obj.falloff, obj.strength, obj.cap, obj.gain,
-                       getattr(obj, "softmax_scale", 0.0))
+                       getattr(obj, "softmax_scale", 0.0), getattr(obj, "extra_gain", ()))
 
 
 def default_params() -> TaraParams:
@@ -177,7 +192,10 @@ def pack_token_meta(segments):
 # device calls (torch tensors in, torch tensors out)
 # ---------------------------------------------------------------------------------------
 class DeviceMeta:
-    """Per-token metadata resident on a device (the four arrays of tara_token_meta)."""
+    """Per-token metadata resident on a device (the arrays of tara_token_meta).
+
+    meta["m_extra"], when present, holds the masks of the extra chained bindings, one row of
+    len(m) weights per binding."""
 
     def __init__(self, meta: dict, device, batch_stride: int = 0, N: Optional[int] = None):
         import torch
@@ -186,6 +204,10 @@ class DeviceMeta:
                                       dtype=torch.float32).to(device)
         self.pic = torch.as_tensor(np.ascontiguousarray(meta["pic"]), dtype=torch.uint8).to(device)
         self.m = torch.as_tensor(np.ascontiguousarray(meta["m"]), dtype=torch.float32).to(device)
+        self.extra_m = None
+        if meta.get("m_extra") is not None and len(meta["m_extra"]) > 0:
+            mx = np.ascontiguousarray(meta["m_extra"], dtype=np.float32).reshape(-1, self.m.numel())
+            self.extra_m = torch.as_tensor(mx).to(device)
         self.batch_stride = int(batch_stride)
         self.N = int(self.seg.numel()) if N is None else int(N)
 
@@ -195,6 +217,10 @@ class DeviceMeta:
         c.pic, c.m = self.pic.data_ptr(), self.m.data_ptr()
         c.N = self.N if N is None else N
         c.batch_stride = self.batch_stride
+        if self.extra_m is not None:
+            c.extra_m, c.extra_m_stride = self.extra_m.data_ptr(), self.extra_m.shape[1]
+        else:
+            c.extra_m, c.extra_m_stride = None, 0
         return c
 
 

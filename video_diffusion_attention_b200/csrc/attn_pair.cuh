@@ -37,10 +37,11 @@ struct PairShape {
                                                       // V half: 128 keys x 64 d (one panel)
   static constexpr int kStages = 8;                   // ring slots (K_j and V_j alternate)
   static constexpr int kKeyBufBytes = 2 * kTile * 16; // [parity][key] float4
+  static constexpr int kRowWBytes = kTile * 17 * 4;   // [row] extra-binding weights
   static constexpr int kXchgBytes = 2 * 2 * kTile * 4 + 2 * kTile * 4;  // max [par][wg][row], sum
   static constexpr int kBarCount = 1 + 2 * kStages + 2 + 2 + 1 + 1 + 1 + 4 + 1;
   static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kHalfBytes + kKeyBufBytes +
-                                    kXchgBytes + kBarCount * 8 + 16;
+                                    kRowWBytes + kXchgBytes + kBarCount * 8 + 16;
   static constexpr uint32_t kColO = 256;
 };
 
@@ -68,7 +69,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + S::kQBytes;
   float4* kbuf = reinterpret_cast<float4*>(sKV + NS * HB);
-  float* xmax = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(kbuf) + S::kKeyBufBytes);
+  float* rowx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(kbuf) + S::kKeyBufBytes);
+  float* xmax = rowx + kTile * 17;
   float* xsum = xmax + 2 * 2 * kTile;
   uint64_t* bars = reinterpret_cast<uint64_t*>(xsum + 2 * kTile);
   uint64_t* q_full = bars;
@@ -233,6 +235,17 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       t_q = args.time_s[mtok + row];
       m_q = args.m[mtok + row];
     }
+    // weights of the extra bindings for this row, one per Picture index (0 for index 0)
+    float* wx = rowx + r * 17;
+    if (bp.n_extra > 0) {
+      for (int pidx = 0; pidx < 16; ++pidx) {
+        float acc = 0.0f;
+        if (is_tgt)
+          for (int k = 0; k < bp.n_extra; ++k)
+            acc += args.xm.m[k * args.xm.stride + mtok + row] * bp.lng_x[k][pidx];
+        wx[pidx] = acc;
+      }
+    }
     TileRec qr;
     if (qtile < args.ntiles) {
       qr = recs[qtile];
@@ -261,7 +274,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       float rowb2 = 0.0f;
       if (is_tgt) {
         if (cls == kClsConstCap) rowb2 = cval * kLog2e;
-        else if (cls == kClsConstPic) rowb2 = (m_q * cval) * kLog2e;
+        else if (cls == kClsConstPic)
+          rowb2 = (bp.n_extra > 0 ? m_q * cval + wx[kr.single_pic & 15] : m_q * cval) * kLog2e;
       }
       float4* kb = kbuf + (j & 1) * kTile;
       if (cls == kClsFull) {
@@ -299,6 +313,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           const float x = fmaxf(fabsf(t_q - kv.x) - w, 0.0f) * inv_f;
           const float pen = fminf(st * (x * x), cap);
           float bb = fmaf(-kv.z, pen, m_q * kv.y);
+          if (bp.n_extra > 0) bb += wx[(int)kv.w];
           bb = is_tgt ? bb : 0.0f;
           s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl, bb * kLog2e));
         }

@@ -14,17 +14,12 @@ constexpr int kSimtRows = 4;     // query rows (warps) per CTA
 constexpr int kSimtChunk = 32;   // keys per shared-memory chunk
 constexpr int kSimtMaxD = 256;
 
-template <typename T>
-__device__ __forceinline__ float to_f32(T x);
-template <>
-__device__ __forceinline__ float to_f32<float>(float x) { return x; }
-
 __global__ void __launch_bounds__(kSimtRows * 32)
 attn_simt_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                  const float* __restrict__ V, float* __restrict__ O, float* __restrict__ LSE,
                  const uint8_t* __restrict__ seg, const float* __restrict__ time_s,
                  const uint8_t* __restrict__ pic, const float* __restrict__ mw,
-                 long long batch_stride, int H, int N, int D, BiasParams bp) {
+                 long long batch_stride, int H, int N, int D, BiasParams bp, ExtraMasks xm) {
   extern __shared__ float smem[];
   const int ld = D + 1;                           // padded row: conflict-free column reads
   float* sK = smem;                               // [chunk][ld]
@@ -80,6 +75,8 @@ attn_simt_kernel(const float* __restrict__ Q, const float* __restrict__ K,
         } else if (sj == kSegPicture) {
           const int pj = pic[mb + j];
           bias = m_q * (pj < 16 ? bp.lng[pj] : 0.0f);
+          for (int k = 0; k < bp.n_extra; ++k)
+            bias += xm.m[k * xm.stride + mb + row] * (pj < 16 ? bp.lng_x[k][pj] : 0.0f);
         }
       }
       x = fmaf(dot, bp.scale_log2, bias * kLog2e);   // log2 units

@@ -46,9 +46,11 @@ struct TcShape {
   static constexpr int kPanelBytes = kTile * 128;           // 128 rows x 128 bytes
   static constexpr int kStages = (D == 128) ? 4 : 8;        // K/V ring slots
   static constexpr int kKeyBufBytes = 2 * 2 * kTile * 16;  // [query tile][parity][key] float4
+  static constexpr int kRowWBytes = 2 * kTile * 17 * 4;     // [tile][row] extra-binding weights
   static constexpr int kBarCount = 1 + 2 * kStages + 2 + 2 + 2 + 1 + 2;
   static constexpr int kSmemBytes = 1024 /*alignment slack*/ + 2 * kTileBytes +
-                                    kStages * kTileBytes + kKeyBufBytes + kBarCount * 8 + 16;
+                                    kStages * kTileBytes + kKeyBufBytes + kRowWBytes +
+                                    kBarCount * 8 + 16;
   static constexpr uint32_t kColS = 0;        // S_t at kColS + 128 t
   static constexpr uint32_t kColO = 256;      // O_t at kColO + D t
   static constexpr uint32_t kColP = 64;       // P_t at S_t + kColP
@@ -67,6 +69,7 @@ struct TcArgs {
   int per_branch_meta;     // 1 when every branch has its own metadata set
   int* status;
   BiasParams bp;
+  ExtraMasks xm;           // masks of chained bindings beyond the first (bp.n_extra of them)
 };
 
 // A wait every lane of the warp leaves together (the tcgen05 loads and stores that follow are
@@ -119,7 +122,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* sQ = smem;                       // 2 tiles
   uint8_t* sKV = smem + 2 * TB;             // NS slots
   float4* kbuf = reinterpret_cast<float4*>(sKV + NS * TB);    // per-key records of full tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * TB + S::kKeyBufBytes);
+  float* rowx = reinterpret_cast<float*>(sKV + NS * TB + S::kKeyBufBytes);   // [tile][row][17]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * TB + S::kKeyBufBytes + S::kRowWBytes);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + NS;
@@ -273,6 +277,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       t_q = args.time_s[mtok + row];
       m_q = args.m[mtok + row];
     }
+    // weights of the extra bindings for this row, one per Picture index (0 for index 0)
+    float* wx = rowx + (t * kTile + r) * 17;
+    if (bp.n_extra > 0) {
+      for (int pidx = 0; pidx < 16; ++pidx) {
+        float acc = 0.0f;
+        if (is_tgt)
+          for (int k = 0; k < bp.n_extra; ++k)
+            acc += args.xm.m[k * args.xm.stride + mtok + row] * bp.lng_x[k][pidx];
+        wx[pidx] = acc;
+      }
+    }
     TileRec qr;
     if (qtile < args.ntiles) {
       qr = recs[qtile];
@@ -302,7 +317,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       float rowb2 = 0.0f;
       if (is_tgt) {
         if (cls == kClsConstCap) rowb2 = cval * kLog2e;
-        else if (cls == kClsConstPic) rowb2 = (m_q * cval) * kLog2e;
+        else if (cls == kClsConstPic)
+          rowb2 = (bp.n_extra > 0 ? m_q * cval + wx[kr.single_pic & 15] : m_q * cval) * kLog2e;
       }
       float4* kb = kbuf + (t * 2 + (j & 1)) * kTile;
       if (cls == kClsFull) {
@@ -334,14 +350,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // rows (a per-element branch on the row role costs ~10x here)
         const float w = bp.window, inv_f = bp.inv_falloff, st = bp.strength, cap = bp.cap;
         const float sl = bp.scale_log2;
+        if (bp.n_extra == 0) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float4 kv = kb[c];
-          const float x = fmaxf(fabsf(t_q - kv.x) - w, 0.0f) * inv_f;
-          const float pen = fminf(st * (x * x), cap);
-          float b = fmaf(-kv.z, pen, m_q * kv.y);
-          b = is_tgt ? b : 0.0f;
-          s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl, b * kLog2e));
+          for (int c = 0; c < 128; ++c) {
+            const float4 kv = kb[c];
+            const float x = fmaxf(fabsf(t_q - kv.x) - w, 0.0f) * inv_f;
+            const float pen = fminf(st * (x * x), cap);
+            float b = fmaf(-kv.z, pen, m_q * kv.y);
+            b = is_tgt ? b : 0.0f;
+            s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl, b * kLog2e));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const float4 kv = kb[c];
+            const float x = fmaxf(fabsf(t_q - kv.x) - w, 0.0f) * inv_f;
+            const float pen = fminf(st * (x * x), cap);
+            float b = fmaf(-kv.z, pen, m_q * kv.y) + wx[(int)kv.w];
+            b = is_tgt ? b : 0.0f;
+            s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl, b * kLog2e));
+          }
         }
         mx = row_max128(s);
         scl = 1.0f;

@@ -86,6 +86,11 @@ int check_params(const tara_params* p) {
     return TARA_ERR_PARAM;
   for (int i = 0; i < 9; ++i)
     if (!finite_f(p->gain[i]) || p->gain[i] <= 0.0f) return TARA_ERR_PARAM;
+  if (p->n_extra_bindings < 0 || p->n_extra_bindings > TARA_MAX_EXTRA_BINDINGS)
+    return TARA_ERR_PARAM;
+  for (int k = 0; k < p->n_extra_bindings; ++k)
+    for (int i = 0; i < 9; ++i)
+      if (!finite_f(p->extra_gain[k][i]) || p->extra_gain[k][i] <= 0.0f) return TARA_ERR_PARAM;
   return TARA_OK;
 }
 
@@ -105,6 +110,12 @@ BiasParams make_bias_params(const tara_params* p, int D) {
     bp.lng[i] = (float)std::log((double)p->gain[i - 1]);
     if (bp.lng[i] != 0.0f) bp.lng_nz |= 1u << i;
   }
+  bp.n_extra = p->n_extra_bindings;
+  for (int k = 0; k < p->n_extra_bindings; ++k)
+    for (int i = 1; i <= 9; ++i) {
+      bp.lng_x[k][i] = (float)std::log((double)p->extra_gain[k][i - 1]);
+      if (bp.lng_x[k][i] != 0.0f) bp.lng_nz |= 1u << i;
+    }
   return bp;
 }
 
@@ -238,7 +249,15 @@ int validate(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
   if ((reinterpret_cast<uintptr_t>(meta->time_s) & 3u) != 0 ||
       (reinterpret_cast<uintptr_t>(meta->m) & 3u) != 0)
     return TARA_ERR_ALIGN;
-  return check_params(p);
+  int rc = check_params(p);
+  if (rc != TARA_OK || p->n_extra_bindings == 0) return rc;
+  // masks of the extra bindings: one array per binding, each as long as m
+  if (!meta->extra_m) return TARA_ERR_NULL;
+  const long long nsets = meta->batch_stride != 0 ? Q->B : 1;
+  const long long m_len = (nsets - 1) * (long long)meta->batch_stride + meta->N;
+  if (meta->extra_m_stride < m_len) return TARA_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(meta->extra_m) & 3u) != 0) return TARA_ERR_ALIGN;
+  return TARA_OK;
 }
 
 }  // namespace
@@ -256,6 +275,9 @@ void tara_default_params(tara_params* p) {
   p->cap = 6.0f;
   for (int i = 0; i < 9; ++i) p->gain[i] = 1.0f;
   p->softmax_scale = 0.0f;
+  p->n_extra_bindings = 0;
+  for (int k = 0; k < TARA_MAX_EXTRA_BINDINGS; ++k)
+    for (int i = 0; i < 9; ++i) p->extra_gain[k][i] = 1.0f;
 }
 
 const char* tara_status_string(int s) {
@@ -303,7 +325,8 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
     attn_simt_kernel<<<grid, kSimtRows * 32, smem, stream>>>(
         static_cast<const float*>(Q->ptr), static_cast<const float*>(K->ptr),
         static_cast<const float*>(V->ptr), static_cast<float*>(O->ptr), LSE, meta->seg,
-        meta->time_s, meta->pic, meta->m, (long long)meta->batch_stride, H, N, D, bp);
+        meta->time_s, meta->pic, meta->m, (long long)meta->batch_stride, H, N, D, bp,
+        ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride});
     if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
     return record_stop(stream);
   }
@@ -343,6 +366,7 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
   a.per_branch_meta = meta->batch_stride != 0 ? 1 : 0;
   a.status = st->status;
   a.bp = bp;
+  a.xm = ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride};
   const bool bf16 = Q->dtype == TARA_BF16;
 #if TARA_PAIR_KERNEL
   if (D == 128)
@@ -523,6 +547,7 @@ extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor
   a.per_branch_meta = meta->batch_stride != 0 ? 1 : 0;
   a.status = st->status;
   a.bp = bp;
+  a.xm = ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride};
   const bool bf16 = Q->dtype == TARA_BF16;
 #if TARA_PAIR_KERNEL
   if (D == 128) {

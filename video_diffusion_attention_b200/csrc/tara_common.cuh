@@ -20,8 +20,16 @@ struct BiasParams {
   float scale;         // softmax scale (natural units)
   float scale_log2;    // softmax scale * log2(e)
   float lng[16];       // ln(gain of Picture p), p = 0..15; 0 for p outside 1..9
-  uint32_t lng_nz;     // bit p set when lng[p] != 0
-  uint32_t pad[3];
+  uint32_t lng_nz;     // bit p set when lng[p] != 0 for any binding
+  int32_t n_extra;     // chained bindings beyond the first (0..3)
+  uint32_t pad[2];
+  float lng_x[3][16];  // ln(gain) of each extra binding
+};
+
+// Extra-binding masks as the kernels see them (token arrays like m, one per binding).
+struct ExtraMasks {
+  const float* m;      // binding k, set b, token i at m[k * stride + b * batch_stride + i]
+  long long stride;
 };
 
 // Summary of one 128-token tile of the packed sequence (written by the tile-summary kernel).
@@ -34,10 +42,11 @@ struct __align__(16) TileRec {
   uint32_t single_pic; // p when every valid token is PICTURE with the same index p, else 0
 };
 
-// Per-key bias record (float4): x = time of a GUIDE key (else 0), y = ln(gain) of a PICTURE
-// key with a non-neutral gain (else 0), z = 1 for a GUIDE key (else 0), w unused.  The bias of
-// the edge (TARGET row with time t and mask m, key) is then -z*penalty(|t - x|) + m*y, with no
-// branch on the key's role.
+// Per-key bias record (float4): x = time of a GUIDE key (else 0), y = ln(gain) of the first
+// binding for a PICTURE key with a non-neutral gain in any binding (else 0), z = 1 for a GUIDE
+// key (else 0), w = its Picture index (else 0).  The bias of the edge (TARGET row with time t
+// and mask m, key) is then -z*penalty(|t - x|) + m*y (+ the row's extra-binding weight of
+// Picture w), with no branch on the key's role.
 
 // Tile-pair classes (per 128-row query tile x 128-key tile).
 constexpr int kClsZero = 0;      // no edge of the pair is biased

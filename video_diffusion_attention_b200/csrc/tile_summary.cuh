@@ -46,8 +46,9 @@ tile_summary_kernel(const uint8_t* __restrict__ seg, const float* __restrict__ t
     if (s == kSegGuide) {
       rec.x = tm;
       rec.z = 1.0f;
-    } else if (s == kSegPicture && pc < 16 && bp.lng[pc] != 0.0f) {
+    } else if (s == kSegPicture && pc < 16 && ((bp.lng_nz >> pc) & 1u)) {
       rec.y = bp.lng[pc];
+      rec.w = (float)pc;
     }
     keyinfo[(long long)set * N + tok] = rec;
   }

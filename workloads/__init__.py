@@ -233,6 +233,32 @@ def make_qkv(w: Workload, device="cpu"):
     return out
 
 
+def chained_masks(w: Workload, n: int, seed: int = 11) -> np.ndarray:
+    """[n][N] float32 masks of n extra chained bindings, in packing order.
+
+    Each binding's mask is a soft ellipse over the target's patch grid (`ellipse_mask` when the
+    frame is 40 x 50 patches, else uniform in [0,1]), the same on every frame; the bindings are
+    drawn independently, so their masks overlap.  Tokens outside TARGET segments get uniform
+    noise: the rule ignores them, and nonzero values there check that it does.
+    """
+    g = np.random.Generator(np.random.PCG64(w.seed(40 + seed)))
+    out = np.empty((n, w.N), np.float32)
+    for k in range(n):
+        row, start = [], 0
+        for s in w.segments:
+            if s.kind == TARGET:
+                if s.tokens_per_frame == 40 * 50:
+                    frame = ellipse_mask(w.seed(50 + seed + k))
+                else:
+                    frame = uniform_mask(w.seed(60 + seed + k) + start, s.tokens_per_frame)
+                row.append(np.tile(frame, s.frames))
+            else:
+                row.append(g.uniform(0.0, 1.0, size=s.length).astype(np.float32))
+            start += s.length
+        out[k] = np.concatenate(row)
+    return out
+
+
 def segment_bounds(w: Workload) -> List[tuple]:
     """(kind, start, end, frames, tokens_per_frame) of every segment, in packing order."""
     out, start = [], 0
