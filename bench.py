@@ -372,7 +372,45 @@ def main():
         mask_line = {"kernel": "target_mask_kernel", "workload": "107x544x928 fp32 pixel mask -> "
                      "%dx40x50 target weights" % tgt[0].frames, "ms": mms, "bound": "hbm",
                      "algorithmic_bytes": mbytes, "achieved_GBs": mbytes / (mms * 1e-3) / 1e9}
+    # the INT8 Q K^T variant of the same forward (Q per token, K per 128-key block, 8-bit
+    # tensor cores for Q K^T, P V in bf16): reported beside the headline, never as it
+    q8_line = None
+    if w.D == 128 and w.dtype in ("bf16", "fp16"):
+        p8 = T.params_from(w.params, qk_int8=1)
+        for _ in range(2):
+            T.attn_forward(q, k, v, meta, p8, O, L, stream)
+        reps = 5
+        kev8 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(reps)]
+        for a, b in kev8:
+            a.record(stream)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(reps):
+            T.set_kernel_events(*kev8[i])
+            T.attn_forward(q, k, v, meta, p8, O, L, stream)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        if T.device_status() != 0:
+            raise SystemExit("INT8 kernel reported a device timeout")
+        q8_step = s0.elapsed_time(s1) / reps
+        q8_kernel = statistics.mean(a.elapsed_time(b) for a, b in kev8)
+        q8_line = {"kernel": "attn_tc_kernel<int8 QK>", "ms_per_step": q8_step,
+                   "value": w.flops / (q8_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+                   "kernel_ms": q8_kernel, "flop_basis": "4*B*H*N^2*D, as the headline",
+                   "gpu_launches_per_step": 4}
     peaks, peak_src = load_peaks()
+    if q8_line is not None:
+        # QK^T (half the FLOP) at the 8-bit peak (2x bf16, the nominal ratio), PV at bf16
+        p16 = float(peaks["bf16_tflops_sustained"])
+        q8_peak = 1.0 / (0.5 / (2.0 * p16) + 0.5 / p16)
+        q8_ach = w.flops / (q8_line["kernel_ms"] * 1e-3) / 1e12
+        q8_line["roofline"] = {"bound": "tensor", "achieved": q8_ach, "peak": q8_peak,
+                               "unit": "TFLOP/s", "frac": q8_ach / q8_peak, "traffic": None,
+                               "peak_kind": "QK^T at 2 x measured sustained bf16 (nominal int8 "
+                                            "ratio), PV at measured sustained bf16 (%s)" % peak_src}
     if mask_line is not None:
         mask_line["peak_GBs"] = float(peaks["hbm_gbs"])
         mask_line["frac"] = mask_line["achieved_GBs"] / float(peaks["hbm_gbs"])
@@ -401,6 +439,8 @@ def main():
     }
     if mask_line is not None:
         line["mask_prep"] = mask_line
+    if q8_line is not None:
+        line["int8_qk"] = q8_line
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, dt, threads = oracle_sample_rate(w, args.cpu_budget, device_inputs=(q, k, v))
         line["cpu_baseline"] = {

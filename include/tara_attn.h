@@ -130,10 +130,17 @@ typedef struct {
    * key of Picture p then get m_i ln(gain[p-1]) + sum_k m_k,i ln(extra_gain[k][p-1]).        */
   int32_t n_extra_bindings;
   float extra_gain[TARA_MAX_EXTRA_BINDINGS][9];
+  /* INT8 QK^T ("TARA: ...", "Three backends": the one-pass kernels run the rule on dense INT8
+   * attention).  0: Q K^T in the inputs' 16-bit type.  1: the library quantises Q per token
+   * and K per 128-token block to symmetric 8-bit codes (tara_quantize_qk_int8) and runs Q K^T
+   * on 8-bit tensor cores; the rule, the softmax and P V are unchanged (P and V 16-bit).
+   * bf16/fp16 with D = 128 only; other values, dtypes or head sizes return TARA_ERR_PARAM,
+   * TARA_ERR_DTYPE, TARA_ERR_HEAD_DIM.                                                     */
+  int32_t qk_int8;
 } tara_params;
 
-/* Fill *p with the defaults above (all gains 1, softmax_scale 0, no extra bindings).  NULL
- * is ignored. */
+/* Fill *p with the defaults above (all gains 1, softmax_scale 0, no extra bindings, 16-bit
+ * QK^T).  NULL is ignored. */
 void tara_default_params(tara_params* p);
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -158,6 +165,26 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
                       const tara_token_meta* meta, const tara_params* p,
                       tara_tensor* O, float* LSE, void* stream);
 
+/* ---- 8-bit quantisation of Q and K ------------------------------------------------------ */
+/* The quantisation tara_attn_forward runs when p->qk_int8 = 1, exposed for callers that keep
+ * the codes ("TARA: ...", "Three backends" names dense INT8 kernels without their scaling;
+ * the scheme below is this library's reading).
+ *   Q, K    : device tensors [B][H][N][D], bf16 or fp16, D = 64 or 128, same shape and dtype,
+ *             finite values, 16-byte aligned.
+ *   q_codes : device int8 [B][H][N][D] (written): Q quantised per token.
+ *   q_scale : device float [B][H][N] (written).
+ *   k_codes : device int8 [B][H][N][D] (written): K quantised per block of 128 consecutive
+ *             tokens of one (branch, head); the last block holds the N % 128 remaining tokens.
+ *   k_scale : device float [B][H][ceil(N/128)] (written).
+ *   stream  : CUDA stream, 0 for the legacy default stream.
+ * Per group: amax = max |x|, inv = 127 / amax, code = rint(x * inv) (float32 product, ties to
+ * even), scale = amax / 127 (IEEE float32 divisions); amax <= 1e-30 gives codes 0, scale 0.
+ * x is approximated by code * scale.  Code arrays 16-byte aligned, scale arrays 4-byte.
+ * Errors: TARA_ERR_NULL, _SHAPE, _DTYPE, _HEAD_DIM, _ALIGN, _TOO_LARGE before any launch;
+ * TARA_ERR_CUDA on a launch failure.                                                       */
+int tara_quantize_qk_int8(const tara_tensor* Q, const tara_tensor* K, int8_t* q_codes,
+                          float* q_scale, int8_t* k_codes, float* k_scale, void* stream);
+
 /* ---- allocation-free variant ------------------------------------------------------------ */
 /* Largest scratch (bytes) tara_attn_forward_noalloc can use: per metadata set, 16 bytes per
  * token plus 32 bytes per 128-token tile (4 MiB covers one shared set of up to ~260,000
@@ -173,7 +200,8 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
  *   - Scratch: a fixed module array of TARA_NOALLOC_SCRATCH_BYTES on each device instead of
  *     the cached workspace; sizes that need more return TARA_ERR_TOO_LARGE before anything
  *     is launched.  fp32 inputs return TARA_ERR_DTYPE (their kernel needs no scratch; call
- *     tara_attn_forward).
+ *     tara_attn_forward); qk_int8 = 1 returns TARA_ERR_PARAM (its 8-bit copies of Q and K
+ *     do not fit the array).
  *   - Set-up: the first call on each device (that device current) looks up the array's device
  *     address with cudaGetSymbolAddress; make that first call before any stream capture.
  *   - Sharing: every call on a device uses the same array and leaves its contents behind;

@@ -22,10 +22,12 @@ def _with_extra(meta: dict, m_extra, copies: int = 1) -> dict:
     return meta
 
 
-def run_gpu(w: W.Workload, q, k, v, per_branch_meta: bool = False, m_extra=None):
+def run_gpu(w: W.Workload, q, k, v, per_branch_meta: bool = False, m_extra=None,
+            qk_int8: int = 0):
     """O, LSE from the CUDA path (through the C ABI) for workload w on cuda tensors q, k, v.
 
-    m_extra: [n][N] masks of the chained bindings named by w.params.extra_gain (or None)."""
+    m_extra: [n][N] masks of the chained bindings named by w.params.extra_gain (or None);
+    qk_int8: 1 runs Q K^T on 8-bit codes."""
     import video_diffusion_attention_b200 as T
     meta = T.pack_token_meta(w.segments)
     if per_branch_meta:
@@ -34,7 +36,7 @@ def run_gpu(w: W.Workload, q, k, v, per_branch_meta: bool = False, m_extra=None)
         dmeta = T.DeviceMeta(_with_extra(stacked, m_extra, w.B), q.device, batch_stride=N, N=N)
     else:
         dmeta = T.DeviceMeta(_with_extra(meta, m_extra), q.device)
-    O, L = T.attn_forward(q, k, v, dmeta, T.params_from(w.params))
+    O, L = T.attn_forward(q, k, v, dmeta, T.params_from(w.params, qk_int8))
     torch.cuda.synchronize()
     assert T.device_status() == 0
     return O, L
@@ -46,6 +48,25 @@ def run_oracle(w: W.Workload, q, k, v, rows: np.ndarray, m_extra=None):
     raw = [oracle.torch_to_numpy_raw(t) for t in (q, k, v)]
     return oracle.attention_rows(raw[0][0], raw[1][0], raw[2][0], raw[0][1], meta, w.params,
                                  rows)
+
+
+def run_oracle_int8(w: W.Workload, q, k, v, rows: np.ndarray, m_extra=None):
+    """O, LSE (fp64) of the INT8-QK^T oracle for rows (b, h, i), one head at a time (the
+    quantisation groups never span heads), in the order of `rows`."""
+    from oracle import int8_qk
+    meta = _with_extra(oracle.pack_token_meta(w.segments), m_extra)
+    raw = [oracle.torch_to_numpy_raw(t) for t in (q, k, v)]
+    dtype = raw[0][1]
+    O = np.empty((rows.shape[0], w.D))
+    L = np.empty((rows.shape[0],))
+    for h in np.unique(rows[:, 1]):
+        sel = np.where(rows[:, 1] == h)[0]
+        sub = [np.ascontiguousarray(r[0][:, h:h + 1]) for r in raw]
+        local = rows[sel].copy()
+        local[:, 1] = 0
+        O[sel], L[sel] = int8_qk.attention_rows_int8qk(sub[0], sub[1], sub[2], dtype, meta,
+                                                       w.params, local)
+    return O, L
 
 
 def rows_from_sample(sample: dict) -> np.ndarray:

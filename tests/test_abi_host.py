@@ -177,6 +177,47 @@ def test_extra_binding_checks(lib):
         B.make_params(extra_gain=((1.0,) * 8,))
 
 
+def test_int8_qk_checks(lib):
+    assert B.default_params().qk_int8 == 0
+    for bad in (2, -1):
+        assert _call(lib, p=B.make_params(qk_int8=bad)) == -5
+    f, s64 = B.TARA_FP32, (1, 2, 300, 64)
+    assert _call(lib, Q=_t(dtype=f), K=_t(dtype=f), V=_t(dtype=f), O=_t(dtype=f),
+                 p=B.make_params(qk_int8=1)) == -3
+    assert _call(lib, Q=_t(shape=s64), K=_t(shape=s64), V=_t(shape=s64), O=_t(shape=s64),
+                 p=B.make_params(qk_int8=1)) == -4
+    p = B.make_params(qk_int8=1)
+    rc = lib.tara_attn_forward_noalloc(ctypes.byref(_t()), ctypes.byref(_t()), ctypes.byref(_t()),
+                                       ctypes.byref(_meta()), ctypes.byref(p), ctypes.byref(_t()),
+                                       ctypes.c_void_p(FAKE), None)
+    assert rc == -5
+
+
+def _quant_call(lib, Q=None, K=None, qc=FAKE, qs=FAKE, kc=FAKE, ks=FAKE):
+    Q = Q if Q is not None else _t()
+    K = K if K is not None else _t()
+    return lib.tara_quantize_qk_int8(ctypes.byref(Q), ctypes.byref(K), ctypes.c_void_p(qc),
+                                     ctypes.c_void_p(qs), ctypes.c_void_p(kc),
+                                     ctypes.c_void_p(ks), None)
+
+
+def test_quantize_argument_checks(lib):
+    assert _quant_call(lib, qc=0) == -1
+    assert _quant_call(lib, ks=0) == -1
+    assert _quant_call(lib, Q=_t(ptr=0)) == -1
+    assert _quant_call(lib, Q=_t(dtype=B.TARA_FP32), K=_t(dtype=B.TARA_FP32)) == -3
+    assert _quant_call(lib, K=_t(dtype=B.TARA_FP16)) == -3
+    assert _quant_call(lib, K=_t(shape=(1, 2, 301, 128))) == -2
+    assert _quant_call(lib, Q=_t(shape=(1, 2, 0, 128)), K=_t(shape=(1, 2, 0, 128))) == -2
+    s96 = (1, 2, 300, 96)
+    assert _quant_call(lib, Q=_t(shape=s96), K=_t(shape=s96)) == -4
+    big = (300, 300, 4, 128)
+    assert _quant_call(lib, Q=_t(shape=big), K=_t(shape=big)) == -11
+    assert _quant_call(lib, kc=FAKE + 8) == -6
+    assert _quant_call(lib, qs=FAKE + 2) == -6
+    assert _quant_call(lib, K=_t(ptr=FAKE + 4)) == -6
+
+
 # ---------------------------------------------------------------------------------------
 # the packer against the oracle's packer (bit-exact) and its error handling
 # ---------------------------------------------------------------------------------------

@@ -14,6 +14,6 @@ marshals arguments.  Build the library with `python -m video_diffusion_attention
 from ._binding import (  # noqa: F401
     DeviceMeta, TaraError, attn_forward, default_params, device_status, load_library,
     make_params, pack_token_meta, packed_length, params_from, prepare_target_mask,
-    selftest_wait, set_kernel_events, SEG_AUDIO, SEG_GUIDE,
+    quantize_qk_int8, selftest_wait, set_kernel_events, SEG_AUDIO, SEG_GUIDE,
     SEG_OTHER_VIDEO, SEG_PICTURE, SEG_TARGET, SEG_TEXT, TARA_BF16, TARA_FP16, TARA_FP32,
 )

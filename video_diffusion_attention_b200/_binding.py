@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = ("tara_default_params", "tara_status_string", "tara_attn_forward",
            "tara_device_status", "tara_packed_length", "tara_pack_token_meta",
            "tara_set_kernel_events", "tara_selftest_wait", "tara_attn_forward_noalloc",
-           "tara_prepare_target_mask")
+           "tara_prepare_target_mask", "tara_quantize_qk_int8")
 
 
 class TaraError(RuntimeError):
@@ -56,7 +56,8 @@ class TaraParams(ctypes.Structure):
                 ("strength", ctypes.c_float), ("cap", ctypes.c_float),
                 ("gain", ctypes.c_float * 9), ("softmax_scale", ctypes.c_float),
                 ("n_extra_bindings", ctypes.c_int32),
-                ("extra_gain", (ctypes.c_float * 9) * MAX_EXTRA_BINDINGS)]
+                ("extra_gain", (ctypes.c_float * 9) * MAX_EXTRA_BINDINGS),
+                ("qk_int8", ctypes.c_int32)]
 
 
 class TaraSegment(ctypes.Structure):
@@ -89,6 +90,8 @@ def load_library(path: Optional[str] = None):
         ctypes.c_void_p, ctypes.c_void_p]
     lib.tara_attn_forward_noalloc.restype = ctypes.c_int
     lib.tara_attn_forward_noalloc.argtypes = lib.tara_attn_forward.argtypes
+    lib.tara_quantize_qk_int8.restype = ctypes.c_int
+    lib.tara_quantize_qk_int8.argtypes = [ctypes.POINTER(TaraTensor)] * 2 + [ctypes.c_void_p] * 5
     lib.tara_set_kernel_events.restype = ctypes.c_int
     lib.tara_set_kernel_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.tara_prepare_target_mask.restype = ctypes.c_int
@@ -112,8 +115,9 @@ def load_library(path: Optional[str] = None):
 # parameters and packing
 # ---------------------------------------------------------------------------------------
 def make_params(window=0.20, falloff=0.25, strength=2.0, cap=6.0, gain=(1.0,) * 9,
-                softmax_scale=0.0, extra_gain=()) -> TaraParams:
-    """TaraParams; extra_gain lists the 9 gains of each chained binding beyond the first."""
+                softmax_scale=0.0, extra_gain=(), qk_int8=0) -> TaraParams:
+    """TaraParams; extra_gain lists the 9 gains of each chained binding beyond the first;
+    qk_int8=1 selects 8-bit Q K^T."""
     p = TaraParams()
     p.window, p.falloff, p.strength, p.cap = window, falloff, strength, cap
     g = list(gain)
@@ -129,14 +133,16 @@ def make_params(window=0.20, falloff=0.25, strength=2.0, cap=6.0, gain=(1.0,) * 
     for k in range(MAX_EXTRA_BINDINGS):
         for i in range(9):
             p.extra_gain[k][i] = extra[k][i] if k < len(extra) else 1.0
+    p.qk_int8 = int(qk_int8)
     return p
 
 
-def params_from(obj) -> TaraParams:
+def params_from(obj, qk_int8: int = 0) -> TaraParams:
     """TaraParams from any object with window, falloff, strength, cap, gain, softmax_scale
     (and optionally extra_gain)."""
     return make_params(obj.window, obj.falloff, obj.strength, obj.cap, obj.gain,
-                       getattr(obj, "softmax_scale", 0.0), getattr(obj, "extra_gain", ()))
+                       getattr(obj, "softmax_scale", 0.0), getattr(obj, "extra_gain", ()),
+                       qk_int8)
 
 
 def default_params() -> TaraParams:
@@ -291,6 +297,28 @@ def attn_forward_noalloc(q, k, v, meta: DeviceMeta, params: TaraParams, out, lse
     if rc != 0:
         raise TaraError(rc, "tara_attn_forward_noalloc")
     return out, lse
+
+
+def quantize_qk_int8(q, k, stream=None):
+    """8-bit codes and scales of Q (per token) and K (per 128-token block), on the device:
+    (q_codes int8 [B][H][N][D], q_scale f32 [B][H][N], k_codes int8 [B][H][N][D],
+    k_scale f32 [B][H][ceil(N/128)])."""
+    import torch
+    B, H, N, D = q.shape
+    qc = torch.empty((B, H, N, D), dtype=torch.int8, device=q.device)
+    kc = torch.empty((B, H, N, D), dtype=torch.int8, device=q.device)
+    qs = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    ks = torch.empty((B, H, (N + 127) // 128), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    cq, ck = tensor_struct(q), tensor_struct(k)
+    rc = load_library().tara_quantize_qk_int8(
+        ctypes.byref(cq), ctypes.byref(ck), ctypes.c_void_p(qc.data_ptr()),
+        ctypes.c_void_p(qs.data_ptr()), ctypes.c_void_p(kc.data_ptr()),
+        ctypes.c_void_p(ks.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise TaraError(rc, "tara_quantize_qk_int8")
+    return qc, qs, kc, ks
 
 
 def prepare_target_mask(mask, shot_len: int, frames_per_latent: int, F_lat: int, Hq: int,

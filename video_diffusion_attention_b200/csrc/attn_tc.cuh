@@ -39,16 +39,18 @@ constexpr int kExpEmuPeriod = TARA_EXP_EMU_PERIOD;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait; a normal wait is microseconds
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s to let in-flight copies/MMAs land
 
-template <int D>
+template <int D, bool kQ8 = false>
 struct TcShape {
   static constexpr int kTileBytes = kTile * D * 2;          // one 128 x D 16-bit tile
+  // Q and K tiles: 16-bit, or 8-bit codes (one 128-byte swizzle panel per row at D = 128)
+  static constexpr int kQKTileBytes = kQ8 ? kTile * D : kTileBytes;
   static constexpr int kPanels = D / 64;                    // 128-byte swizzle panels per row
   static constexpr int kPanelBytes = kTile * 128;           // 128 rows x 128 bytes
   static constexpr int kStages = (D == 128) ? 4 : 8;        // K/V ring slots
   static constexpr int kKeyBufBytes = 2 * 2 * kTile * 16;  // [query tile][parity][key] float4
   static constexpr int kRowWBytes = 2 * kTile * 17 * 4;     // [tile][row] extra-binding weights
   static constexpr int kBarCount = 1 + 2 * kStages + 2 + 2 + 2 + 1 + 2;
-  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + 2 * kTileBytes +
+  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + 2 * kQKTileBytes +
                                     kStages * kTileBytes + kKeyBufBytes + kRowWBytes +
                                     kBarCount * 8 + 16;
   static constexpr uint32_t kColS = 0;        // S_t at kColS + 128 t
@@ -70,6 +72,8 @@ struct TcArgs {
   int* status;
   BiasParams bp;
   ExtraMasks xm;           // masks of chained bindings beyond the first (bp.n_extra of them)
+  const float* q_scale;    // INT8 QK^T: per-token Q scales [B*H][N]
+  const float* k_scale;    // INT8 QK^T: per-key-tile K scales [B*H][ntiles]
 };
 
 // A wait every lane of the warp leaves together (the tcgen05 loads and stores that follow are
@@ -108,19 +112,24 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
   return kBF16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
 }
 
-template <bool kBF16, int D>
+// kQ8: Q and K arrive as 8-bit codes (tmQ, tmK map the code arrays), QK^T runs as
+// tcgen05.mma.kind::i8 into an s32 S, and the softmax scales row i of key tile j by
+// q_scale[i] * k_scale[j]; P and V stay 16-bit.
+template <bool kBF16, int D, bool kQ8 = false>
 __global__ void __launch_bounds__(384, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const TcArgs args) {
-  using S = TcShape<D>;
+  static_assert(!kQ8 || D == 128, "8-bit Q/K tiles use one 128-byte panel per row");
+  using S = TcShape<D, kQ8>;
   constexpr int TB = S::kTileBytes;
+  constexpr int QKB = S::kQKTileBytes;
   constexpr int NS = S::kStages;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                       // 2 tiles
-  uint8_t* sKV = smem + 2 * TB;             // NS slots
+  uint8_t* sKV = smem + 2 * QKB;            // NS slots
   float4* kbuf = reinterpret_cast<float4*>(sKV + NS * TB);    // per-key records of full tiles
   float* rowx = reinterpret_cast<float*>(sKV + NS * TB + S::kKeyBufBytes);   // [tile][row][17]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * TB + S::kKeyBufBytes + S::kRowWBytes);
@@ -177,20 +186,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * TB);
-      for (int t = 0; t < 2; ++t)
-        for (int p = 0; p < S::kPanels; ++p)
-          tma_load_3d(sQ + t * TB + p * S::kPanelBytes, &tmQ, q_full, p * 64, (qt0 + t) * kTile, bh);
+      mbar_arrive_expect_tx(q_full, 2 * QKB);
+      for (int t = 0; t < 2; ++t) {
+        if (kQ8) {
+          tma_load_3d(sQ + t * QKB, &tmQ, q_full, 0, (qt0 + t) * kTile, bh);
+        } else {
+          for (int p = 0; p < S::kPanels; ++p)
+            tma_load_3d(sQ + t * TB + p * S::kPanelBytes, &tmQ, q_full, p * 64, (qt0 + t) * kTile, bh);
+        }
+      }
       int issued = 0;
       for (int i = 0; i < 2 * nk; ++i) {
         const int slot = i % NS;
         const uint32_t ph = (uint32_t)(i / NS) & 1u;
         if (!mbar_wait(&kv_empty[slot], ph ^ 1u, abort_flag, kWaitLimitNs)) break;
-        mbar_arrive_expect_tx(&kv_full[slot], TB);
-        const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
-        for (int p = 0; p < S::kPanels; ++p)
-          tma_load_3d(sKV + slot * TB + p * S::kPanelBytes, map, &kv_full[slot], p * 64,
-                      (i >> 1) * kTile, bh);
+        if (kQ8 && !(i & 1)) {
+          mbar_arrive_expect_tx(&kv_full[slot], QKB);
+          tma_load_3d(sKV + slot * TB, &tmK, &kv_full[slot], 0, (i >> 1) * kTile, bh);
+        } else {
+          mbar_arrive_expect_tx(&kv_full[slot], TB);
+          const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+          for (int p = 0; p < S::kPanels; ++p)
+            tma_load_3d(sKV + slot * TB + p * S::kPanelBytes, map, &kv_full[slot], p * 64,
+                        (i >> 1) * kTile, bh);
+        }
         issued = i + 1;
       }
       if (*abort_flag) {
@@ -202,7 +221,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     } else if (warp == 9 && lane == 0) {
       // ------------------------------ MMA issuer --------------------------------
-      constexpr uint32_t idesc_qk = make_idesc_f16(128, 128, kBF16, false);
+      constexpr uint32_t idesc_qk = kQ8 ? make_idesc_s8(128, 128) : make_idesc_f16(128, 128, kBF16, false);
       constexpr uint32_t idesc_pv = make_idesc_f16(128, D, kBF16, true);
       const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
       // base descriptors; a byte offset moves the start-address field by offset >> 4 (shared
@@ -238,12 +257,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           if (j < nk) {
             const uint32_t d_s = tmem + S::kColS + t * 128;
-            const uint64_t qd = qd0 + (uint64_t)((t * TB) >> 4);
+            const uint64_t qd = qd0 + (uint64_t)((t * QKB) >> 4);
             const uint64_t kd = kd0 + (uint64_t)((kslot * TB) >> 4);
+            if (kQ8) {
+              // 32 one-byte codes per instruction: K-steps of 32 bytes along the single panel
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t off = (uint64_t)((((kk >> 2) * S::kPanelBytes) + (kk & 3) * 32) >> 4);
-              umma_ss(d_s, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < D / 32; ++kk)
+                umma_ss_i8(d_s, qd + (uint64_t)((kk * 32) >> 4), kd + (uint64_t)((kk * 32) >> 4),
+                           idesc_qk, kk > 0 ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t off = (uint64_t)((((kk >> 2) * S::kPanelBytes) + (kk & 3) * 32) >> 4);
+                umma_ss(d_s, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+              }
             }
             umma_commit(&s_full[t]);
             if (t == 1) umma_commit(&kv_empty[kslot]);
@@ -277,6 +304,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       t_q = args.time_s[mtok + row];
       m_q = args.m[mtok + row];
     }
+    // logit scale in log2 units; with 8-bit Q/K it also carries the row's and the key tile's
+    // dequantisation scales
+    const float row_sl = kQ8 ? bp.scale_log2 * (row_ok ? args.q_scale[(long long)bh * N + row] : 0.0f)
+                             : bp.scale_log2;
+    const float* kscale = args.k_scale + (long long)bh * args.ntiles;
+    float ks_next = kQ8 ? kscale[0] : 1.0f;
     // weights of the extra bindings for this row, one per Picture index (0 for index 0)
     float* wx = rowx + (t * kTile + r) * 17;
     if (bp.n_extra > 0) {
@@ -312,6 +345,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int j = 0; j < nk; ++j) {
       const TileRec kr = kr_next;
       if (j + 1 < nk) kr_next = recs[j + 1];   // in flight while this tile is processed
+      float sl = row_sl;
+      if (kQ8) {
+        // a zero scale (an all-zero Q row or K tile, whose codes are all 0) is raised to the
+        // smallest normal float: valid logits stay exactly 0 and the -inf of masked columns
+        // stays -inf instead of becoming 0 * -inf
+        sl = fmaxf(row_sl * ks_next, 1.17549435e-38f);
+        if (j + 1 < nk) ks_next = kscale[j + 1];
+      }
       float cval;
       const int cls = classify_pair(qr, kr, bp, &cval);
       float rowb2 = 0.0f;
@@ -338,6 +379,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_ld_wait();
       reg_fence<128>(s);
+      if (kQ8) {
+        // s32 dot products of 8-bit codes: |S| <= 127 * 127 * 128 < 2^22, converted exactly
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __float_as_uint(i32_to_f32_small(s[c]));
+      }
       const int nv = (int)kr.nvalid;
       if (nv < kTile) {
 #pragma unroll
@@ -349,7 +395,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // branch-free per-edge bias: computed for every row, zeroed by a select on non-target
         // rows (a per-element branch on the row role costs ~10x here)
         const float w = bp.window, inv_f = bp.inv_falloff, st = bp.strength, cap = bp.cap;
-        const float sl = bp.scale_log2;
         if (bp.n_extra == 0) {
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
@@ -375,8 +420,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         scl = 1.0f;
         off_base = 0.0f;
       } else {
-        mx = fmaf(row_max128(s), bp.scale_log2, rowb2);
-        scl = bp.scale_log2;
+        mx = fmaf(row_max128(s), sl, rowb2);
+        scl = sl;
         off_base = rowb2;
       }
       const float m_new = fmaxf(m_run, mx);

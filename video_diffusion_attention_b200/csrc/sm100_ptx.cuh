@@ -121,6 +121,17 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// D(tmem, s32) (+)= A(smem desc, s8) * B(smem desc, s8)^T; K = 32 per instruction.
+__device__ __forceinline__ void umma_ss_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D(tmem) (+)= A(tmem) * B(smem desc)
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                         uint32_t idesc, uint32_t accumulate) {
@@ -147,6 +158,19 @@ __host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N, bool bf16, b
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::i8: signed 8-bit A and B, s32 accumulator (D format 2).
+__host__ __device__ constexpr uint32_t make_idesc_s8(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+// Exact float value of an int32 with |v| < 2^22: placed in the mantissa of 1.5 * 2^23 (where
+// the float spacing is 1) by an integer add, then the offset is subtracted exactly.  Two
+// full-rate ALU operations instead of one conversion.
+__device__ __forceinline__ float i32_to_f32_small(uint32_t v) {
+  return __uint_as_float(v + 0x4B400000u) - 12582912.0f;
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, tcgen05 version field = 1.

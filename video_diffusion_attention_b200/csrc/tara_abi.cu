@@ -12,6 +12,7 @@
 #include "attn_simt.cuh"
 #include "attn_pair.cuh"
 #include "attn_tc.cuh"
+#include "quant_int8.cuh"
 #include "target_mask.cuh"
 #include "tile_summary.cuh"
 
@@ -35,6 +36,7 @@ struct DeviceState {
   size_t ws_bytes = 0;
   int* status = nullptr;        // device address of g_device_status
   bool tc_attr_set[2][2] = {{false, false}, {false, false}};   // [bf16][D==128]
+  bool tc_q8_attr_set[2] = {false, false};                     // [bf16], D = 128
   bool pair_attr_set[2] = {false, false};                      // [bf16]
   bool simt_attr_set = false;
 };
@@ -91,6 +93,7 @@ int check_params(const tara_params* p) {
   for (int k = 0; k < p->n_extra_bindings; ++k)
     for (int i = 0; i < 9; ++i)
       if (!finite_f(p->extra_gain[k][i]) || p->extra_gain[k][i] <= 0.0f) return TARA_ERR_PARAM;
+  if (p->qk_int8 != 0 && p->qk_int8 != 1) return TARA_ERR_PARAM;
   return TARA_OK;
 }
 
@@ -131,6 +134,50 @@ int encode_qkv_map(CUtensorMap* map, const tara_tensor* t, uint32_t box_rows = k
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? TARA_OK : TARA_ERR_CUDA;
+}
+
+// Tensor map of 8-bit codes [B*H][N][D] (D = 128): one 128-byte swizzle panel per row.
+int encode_q8_map(CUtensorMap* map, const void* codes, int BH, int N, int D) {
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)N * (cuuint64_t)D};
+  const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)kTile, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(codes), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TARA_OK : TARA_ERR_CUDA;
+}
+
+// Quantises Q per token and K per 128-token block (quant_int8.cuh).
+int launch_quant(const tara_tensor* Q, const tara_tensor* K, int8_t* qc, float* qs, int8_t* kc,
+                 float* ks, cudaStream_t stream) {
+  const bool bf16 = Q->dtype == TARA_BF16;
+  const int BH = Q->B * Q->H, N = Q->N, D = Q->D;
+  const long long rows = (long long)BH * N;
+  const unsigned qgrid = (unsigned)((rows + (kQ8Threads / 32) - 1) / (kQ8Threads / 32));
+  const dim3 kgrid((unsigned)((N + kQ8Block - 1) / kQ8Block), (unsigned)BH);
+  const int nb = (N + kQ8Block - 1) / kQ8Block;
+  const uint16_t* q = static_cast<const uint16_t*>(Q->ptr);
+  const uint16_t* k = static_cast<const uint16_t*>(K->ptr);
+  if (D == 128) {
+    if (bf16) {
+      quant_q_kernel<true, 128><<<qgrid, kQ8Threads, 0, stream>>>(q, rows, qc, qs);
+      quant_k_kernel<true, 128><<<kgrid, kQ8Threads, 0, stream>>>(k, N, nb, kc, ks);
+    } else {
+      quant_q_kernel<false, 128><<<qgrid, kQ8Threads, 0, stream>>>(q, rows, qc, qs);
+      quant_k_kernel<false, 128><<<kgrid, kQ8Threads, 0, stream>>>(k, N, nb, kc, ks);
+    }
+  } else {
+    if (bf16) {
+      quant_q_kernel<true, 64><<<qgrid, kQ8Threads, 0, stream>>>(q, rows, qc, qs);
+      quant_k_kernel<true, 64><<<kgrid, kQ8Threads, 0, stream>>>(k, N, nb, kc, ks);
+    } else {
+      quant_q_kernel<false, 64><<<qgrid, kQ8Threads, 0, stream>>>(q, rows, qc, qs);
+      quant_k_kernel<false, 64><<<kgrid, kQ8Threads, 0, stream>>>(k, N, nb, kc, ks);
+    }
+  }
+  return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
 }
 
 // Returns the device's state with a workspace of at least `bytes` (grown with cudaMalloc).
@@ -179,20 +226,21 @@ __global__ void wait_selftest_kernel(int* status, uint64_t limit_ns, int arrive)
   }
 }
 
-template <bool kBF16, int D>
+template <bool kBF16, int D, bool kQ8 = false>
 int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
               const TcArgs& a, int B, int H, int ntiles, cudaStream_t stream, DeviceState* st) {
-  constexpr int smem = TcShape<D>::kSmemBytes;
-  bool& attr = st->tc_attr_set[kBF16 ? 1 : 0][D == 128 ? 1 : 0];
+  constexpr int smem = TcShape<D, kQ8>::kSmemBytes;
+  bool& attr = kQ8 ? st->tc_q8_attr_set[kBF16 ? 1 : 0]
+                   : st->tc_attr_set[kBF16 ? 1 : 0][D == 128 ? 1 : 0];
   if (!attr) {
-    if (cudaFuncSetAttribute(attn_tc_kernel<kBF16, D>,
+    if (cudaFuncSetAttribute(attn_tc_kernel<kBF16, D, kQ8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return TARA_ERR_CUDA;
     attr = true;
   }
   dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
   if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
-  attn_tc_kernel<kBF16, D><<<grid, 384, smem, stream>>>(mq, mk, mv, a);
+  attn_tc_kernel<kBF16, D, kQ8><<<grid, 384, smem, stream>>>(mq, mk, mv, a);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
   return record_stop(stream);
 }
@@ -250,7 +298,12 @@ int validate(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
       (reinterpret_cast<uintptr_t>(meta->m) & 3u) != 0)
     return TARA_ERR_ALIGN;
   int rc = check_params(p);
-  if (rc != TARA_OK || p->n_extra_bindings == 0) return rc;
+  if (rc != TARA_OK) return rc;
+  if (p->qk_int8) {
+    if (Q->dtype == TARA_FP32) return TARA_ERR_DTYPE;
+    if (Q->D != 128) return TARA_ERR_HEAD_DIM;
+  }
+  if (p->n_extra_bindings == 0) return TARA_OK;
   // masks of the extra bindings: one array per binding, each as long as m
   if (!meta->extra_m) return TARA_ERR_NULL;
   const long long nsets = meta->batch_stride != 0 ? Q->B : 1;
@@ -278,6 +331,7 @@ void tara_default_params(tara_params* p) {
   p->n_extra_bindings = 0;
   for (int k = 0; k < TARA_MAX_EXTRA_BINDINGS; ++k)
     for (int i = 0; i < 9; ++i) p->extra_gain[k][i] = 1.0f;
+  p->qk_int8 = 0;
 }
 
 const char* tara_status_string(int s) {
@@ -336,15 +390,33 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
   const int nsets = meta->batch_stride != 0 ? B : 1;
   const size_t rec_bytes = round_up((size_t)nsets * ntiles * sizeof(TileRec), 256);
   const size_t key_bytes = round_up((size_t)nsets * N * sizeof(float4), 256);
+  // 8-bit copies of Q and K with their scales (qk_int8 only)
+  const bool q8 = p->qk_int8 != 0;
+  const size_t code_bytes = q8 ? round_up((size_t)B * H * N * D, 256) : 0;
+  const size_t qs_bytes = q8 ? round_up((size_t)B * H * N * sizeof(float), 256) : 0;
+  const size_t ks_bytes = q8 ? round_up((size_t)B * H * ntiles * sizeof(float), 256) : 0;
   DeviceState* st = nullptr;
-  if ((rc = device_state(rec_bytes + key_bytes, &st)) != TARA_OK) return rc;
-  TileRec* recs = static_cast<TileRec*>(st->ws);
-  float4* keyinfo = reinterpret_cast<float4*>(static_cast<char*>(st->ws) + rec_bytes);
+  if ((rc = device_state(rec_bytes + key_bytes + 2 * code_bytes + qs_bytes + ks_bytes, &st)) !=
+      TARA_OK)
+    return rc;
+  char* ws = static_cast<char*>(st->ws);
+  TileRec* recs = reinterpret_cast<TileRec*>(ws);
+  float4* keyinfo = reinterpret_cast<float4*>(ws + rec_bytes);
+  int8_t* qc = reinterpret_cast<int8_t*>(ws + rec_bytes + key_bytes);
+  int8_t* kc = qc + code_bytes;
+  float* qs = reinterpret_cast<float*>(ws + rec_bytes + key_bytes + 2 * code_bytes);
+  float* ks = reinterpret_cast<float*>(ws + rec_bytes + key_bytes + 2 * code_bytes + qs_bytes);
 
   CUtensorMap mq, mk, mv;
-  if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K) != TARA_OK ||
-      encode_qkv_map(&mv, V) != TARA_OK)
+  if (q8) {
+    if (encode_q8_map(&mq, qc, B * H, N, D) != TARA_OK ||
+        encode_q8_map(&mk, kc, B * H, N, D) != TARA_OK || encode_qkv_map(&mv, V) != TARA_OK)
+      return TARA_ERR_CUDA;
+    if ((rc = launch_quant(Q, K, qc, qs, kc, ks, stream)) != TARA_OK) return rc;
+  } else if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K) != TARA_OK ||
+             encode_qkv_map(&mv, V) != TARA_OK) {
     return TARA_ERR_CUDA;
+  }
 
   tile_summary_kernel<<<dim3((unsigned)ntiles, (unsigned)nsets), 128, 0, stream>>>(
       meta->seg, meta->time_s, meta->pic, N, (long long)meta->batch_stride, ntiles, bp, recs,
@@ -367,7 +439,12 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
   a.status = st->status;
   a.bp = bp;
   a.xm = ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride};
+  a.q_scale = qs;
+  a.k_scale = ks;
   const bool bf16 = Q->dtype == TARA_BF16;
+  if (q8)
+    return bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
+                : launch_tc<false, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st);
 #if TARA_PAIR_KERNEL
   if (D == 128)
     return bf16 ? launch_pair<true>(Q, K, V, a, B, H, ntiles, stream, &st->pair_attr_set[1])
@@ -379,6 +456,25 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
 #endif
   return bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
               : launch_tc<false, 64>(mq, mk, mv, a, B, H, ntiles, stream, st);
+}
+
+int tara_quantize_qk_int8(const tara_tensor* Q, const tara_tensor* K, int8_t* q_codes,
+                          float* q_scale, int8_t* k_codes, float* k_scale, void* stream) {
+  if (!Q || !K || !q_codes || !q_scale || !k_codes || !k_scale) return TARA_ERR_NULL;
+  if (!Q->ptr || !K->ptr) return TARA_ERR_NULL;
+  if (Q->dtype != TARA_BF16 && Q->dtype != TARA_FP16) return TARA_ERR_DTYPE;
+  if (K->dtype != Q->dtype) return TARA_ERR_DTYPE;
+  if (Q->B < 1 || Q->H < 1 || Q->N < 1 || Q->D < 1) return TARA_ERR_SHAPE;
+  if (K->B != Q->B || K->H != Q->H || K->N != Q->N || K->D != Q->D) return TARA_ERR_SHAPE;
+  if (Q->D != 64 && Q->D != 128) return TARA_ERR_HEAD_DIM;
+  if ((long long)Q->B * Q->H > 65535) return TARA_ERR_TOO_LARGE;
+  if (!aligned16(Q->ptr) || !aligned16(K->ptr) || !aligned16(q_codes) || !aligned16(k_codes))
+    return TARA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(q_scale) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(k_scale) & 3u) != 0)
+    return TARA_ERR_ALIGN;
+  return launch_quant(Q, K, q_codes, q_scale, k_codes, k_scale,
+                      static_cast<cudaStream_t>(stream));
 }
 
 int tara_set_kernel_events(void* start, void* stop) {
@@ -505,6 +601,7 @@ extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor
   int rc = validate(Q, K, V, meta, p, O, LSE);
   if (rc != TARA_OK) return rc;
   if (Q->dtype == TARA_FP32) return TARA_ERR_DTYPE;   // the fp32 kernel needs no scratch
+  if (p->qk_int8) return TARA_ERR_PARAM;              // 8-bit Q/K copies do not fit the scratch
   const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
   const int ntiles = (N + kTile - 1) / kTile;
   const size_t nsets = meta->batch_stride != 0 ? (size_t)B : 1;
@@ -548,6 +645,8 @@ extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor
   a.status = st->status;
   a.bp = bp;
   a.xm = ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride};
+  a.q_scale = nullptr;
+  a.k_scale = nullptr;
   const bool bf16 = Q->dtype == TARA_BF16;
 #if TARA_PAIR_KERNEL
   if (D == 128) {
