@@ -29,12 +29,16 @@
 
 namespace tara {
 
-// One pair of exponentials in every kExpEmuPeriod is evaluated with exp2_poly on the FMA pipe
-// instead of MUFU (0 disables the split).
-#ifndef TARA_EXP_EMU_PERIOD
-#define TARA_EXP_EMU_PERIOD 0
-#endif
-constexpr int kExpEmuPeriod = TARA_EXP_EMU_PERIOD;
+constexpr int kTcThreads = 384;
+// setmaxnreg split: the launch gives every thread kTcLaunchRegs; the two softmax warpgroups
+// raise theirs to kTcSoftmaxRegs, the control warpgroup lowers its own to kTcControlRegs.  The
+// sum must equal the launch pool, or the raise would wait for registers that never come; the
+// host refuses to launch when ptxas gave the kernel a different register count.
+constexpr int kTcLaunchRegs = 168;
+constexpr int kTcSoftmaxRegs = 176;
+constexpr int kTcControlRegs = 152;
+static_assert(2 * 128 * kTcSoftmaxRegs + 128 * kTcControlRegs == kTcThreads * kTcLaunchRegs,
+              "register split must use the launch pool exactly");
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait; a normal wait is microseconds
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s to let in-flight copies/MMAs land
@@ -84,15 +88,20 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-// Max of the 128 values of a row, as eight independent chains and a final tree.
+// Max of the 128 values of a row: eight independent chains of three-input max, then a tree.
 __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
   float a[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(s[i]);
 #pragma unroll
-  for (int c = 8; c < 128; ++c) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(s[c]));
-  return fmaxf(fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])),
-               fmaxf(fmaxf(a[4], a[5]), fmaxf(a[6], a[7])));
+  for (int c = 8; c < 120; c += 16) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      a[i] = fmax3(a[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], __uint_as_float(s[120 + i]));
+  return fmaxf(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], fmax3(a[5], a[6], a[7])));
 }
 
 // Bounded rendezvous of the warps counted by `bar` (lane 0 of each warp arrives; every lane
@@ -116,7 +125,7 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
 // tcgen05.mma.kind::i8 into an s32 S, and the softmax scales row i of key tile j by
 // q_scale[i] * k_scale[j]; P and V stay 16-bit.
 template <bool kBF16, int D, bool kQ8 = false>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const TcArgs args) {
   static_assert(!kQ8 || D == 128, "8-bit Q/K tiles use one 128-byte panel per row");
@@ -180,7 +189,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 152;\n" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kTcControlRegs) : "memory");
     if (warp == 8 && lane == 0) {
       // ------------------------------ TMA producer ------------------------------
       tma_prefetch_desc(&tmQ);
@@ -283,7 +292,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_wait(drain, 0, &no_abort, kDrainLimitNs);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kTcSoftmaxRegs) : "memory");
     // ------------------------------ softmax warps -------------------------------
     const int t = warp >> 2;            // query tile of this warpgroup
     const int wq = warp & 3;            // TMEM lane quarter
@@ -431,7 +440,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float alpha = ex2_approx(m_run - m_use);   // 1 when not raised, 0 on the first tile
       l_run *= alpha;
       const float off = off_base - m_use;
-      float lsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      // columns in pairs: one packed FMA forms both exponents, one packed add accumulates
+      // both probabilities (two accumulators break the dependency chain)
+      const uint64_t scl2 = f32x2_pack(scl, scl), off2 = f32x2_pack(off, off);
+      uint64_t lsum2[2] = {0ull, 0ull};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         // 64 columns at a time: their P (32 packed words) is stored while the next half runs
@@ -439,19 +451,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int c2 = 0; c2 < 64; c2 += 2) {
           const int c = half * 64 + c2;
-          // every kExpEmuPeriod-th pair of exponentials runs on the FMA pipe
-          const bool emu = kExpEmuPeriod > 0 && ((c >> 1) % (kExpEmuPeriod > 0 ? kExpEmuPeriod : 1)) ==
-                                                    (kExpEmuPeriod > 0 ? kExpEmuPeriod - 1 : 0);
-          const float x0 = fmaf(__uint_as_float(s[c]), scl, off);
-          const float x1 = fmaf(__uint_as_float(s[c + 1]), scl, off);
-          const float p0 = emu ? exp2_poly(x0) : ex2_approx(x0);
-          const float p1 = emu ? exp2_poly(x1) : ex2_approx(x1);
-          lsum[(c >> 1) & 3] += p0 + p1;
+          float x0, x1;
+          f32x2_unpack(f32x2_fma(f32x2_pack_bits(s[c], s[c + 1]), scl2, off2), x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          lsum2[(c >> 1) & 1] = f32x2_add(lsum2[(c >> 1) & 1], f32x2_pack(p0, p1));
           pk[c2 >> 1] = pack_p<kBF16>(p0, p1);
         }
         tmem_st32(tP + half * 32, pk);
       }
-      l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+      {
+        float a0, a1;
+        f32x2_unpack(f32x2_add(lsum2[0], lsum2[1]), a0, a1);
+        l_run += a0 + a1;
+      }
       if (j > 0 && warp_need) {
         // rescale this warp's O rows once the previous PV has landed
         if (!(ok = warp_wait(&pv_done[t], (uint32_t)(j - 1) & 1u, abort_flag, kWaitLimitNs))) break;

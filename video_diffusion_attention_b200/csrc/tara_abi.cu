@@ -149,6 +149,16 @@ int encode_q8_map(CUtensorMap* map, const void* codes, int BH, int N, int D) {
   return r == CUDA_SUCCESS ? TARA_OK : TARA_ERR_CUDA;
 }
 
+// The tensor-core kernel's setmaxnreg split assumes ptxas gave it exactly kTcLaunchRegs
+// registers per thread (the pool the raise draws on); any other count is refused here rather
+// than launched.
+template <typename F>
+int tc_register_check(F* kernel) {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return TARA_ERR_CUDA;
+  return fa.numRegs == kTcLaunchRegs ? TARA_OK : TARA_ERR_CUDA;
+}
+
 // Quantises Q per token and K per 128-token block (quant_int8.cuh).
 int launch_quant(const tara_tensor* Q, const tara_tensor* K, int8_t* qc, float* qs, int8_t* kc,
                  float* ks, cudaStream_t stream) {
@@ -233,6 +243,7 @@ int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& m
   bool& attr = kQ8 ? st->tc_q8_attr_set[kBF16 ? 1 : 0]
                    : st->tc_attr_set[kBF16 ? 1 : 0][D == 128 ? 1 : 0];
   if (!attr) {
+    if (tc_register_check(attn_tc_kernel<kBF16, D, kQ8>) != TARA_OK) return TARA_ERR_CUDA;
     if (cudaFuncSetAttribute(attn_tc_kernel<kBF16, D, kQ8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return TARA_ERR_CUDA;
@@ -240,7 +251,7 @@ int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& m
   }
   dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
   if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
-  attn_tc_kernel<kBF16, D, kQ8><<<grid, 384, smem, stream>>>(mq, mk, mv, a);
+  attn_tc_kernel<kBF16, D, kQ8><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, a);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
   return record_stop(stream);
 }
@@ -582,11 +593,12 @@ template <bool kBF16, int D>
 int launch_tc_static(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const TcArgs& a, int B, int H, int ntiles, cudaStream_t stream) {
   constexpr int smem = TcShape<D>::kSmemBytes;
+  if (tc_register_check(attn_tc_kernel<kBF16, D>) != TARA_OK) return TARA_ERR_CUDA;
   if (cudaFuncSetAttribute(attn_tc_kernel<kBF16, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return TARA_ERR_CUDA;
   dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
-  attn_tc_kernel<kBF16, D><<<grid, 384, smem, stream>>>(mq, mk, mv, a);
+  attn_tc_kernel<kBF16, D><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
 }
 
