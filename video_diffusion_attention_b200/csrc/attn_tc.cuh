@@ -445,12 +445,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t scl2 = f32x2_pack(scl, scl), off2 = f32x2_pack(off, off);
       uint64_t lsum2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        // 64 columns at a time: their P (32 packed words) is stored while the next half runs
-        uint32_t pk[32];
+      for (int qtr = 0; qtr < 4; ++qtr) {
+        // 32 columns at a time: their P (16 packed words) is stored while the next quarter
+        // runs (a small P buffer leaves registers for more exponentials in flight)
+        uint32_t pk[16];
 #pragma unroll
-        for (int c2 = 0; c2 < 64; c2 += 2) {
-          const int c = half * 64 + c2;
+        for (int c2 = 0; c2 < 32; c2 += 2) {
+          const int c = qtr * 32 + c2;
           float x0, x1;
           f32x2_unpack(f32x2_fma(f32x2_pack_bits(s[c], s[c + 1]), scl2, off2), x0, x1);
           const float p0 = ex2_approx(x0);
@@ -458,7 +459,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           lsum2[(c >> 1) & 1] = f32x2_add(lsum2[(c >> 1) & 1], f32x2_pack(p0, p1));
           pk[c2 >> 1] = pack_p<kBF16>(p0, p1);
         }
-        tmem_st32(tP + half * 32, pk);
+        tmem_st16(tP + qtr * 16, pk);
       }
       {
         float a0, a1;
