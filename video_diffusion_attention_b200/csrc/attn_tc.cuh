@@ -116,6 +116,16 @@ __device__ __forceinline__ bool warp_rendezvous(uint64_t* bar, uint32_t& phase,
   return ok;
 }
 
+// Max of 128 signed 32-bit values (the 8-bit path's integer scores).
+__device__ __forceinline__ int row_max128_s32(const uint32_t (&s)[128]) {
+  int a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = (int)s[i];
+#pragma unroll
+  for (int c = 8; c < 128; ++c) a[c & 7] = max(a[c & 7], (int)s[c]);
+  return max(max(max(a[0], a[1]), max(a[2], a[3])), max(max(a[4], a[5]), max(a[6], a[7])));
+}
+
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
   return kBF16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
@@ -388,12 +398,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_ld_wait();
       reg_fence<128>(s);
-      if (kQ8) {
-        // s32 dot products of 8-bit codes: |S| <= 127 * 127 * 128 < 2^22, converted exactly
+      const int nv = (int)kr.nvalid;
+      // 8-bit path: S holds s32 dot products of the codes, |S| <= 127 * 127 * 128 < 2^22.  On
+      // full-width tiles without per-edge bias they stay integers: the row max is an integer
+      // max, and the exponent loop converts them inside its FMA (the integer add places S in
+      // the mantissa of 1.5 * 2^23, whose offset is folded into the FMA's addend).  Other
+      // tiles are converted exactly up front.
+      const bool s_int = kQ8 && nv == kTile && cls != kClsFull;
+      if (kQ8 && !s_int) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = __float_as_uint(i32_to_f32_small(s[c]));
       }
-      const int nv = (int)kr.nvalid;
       if (nv < kTile) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
@@ -429,7 +444,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         scl = 1.0f;
         off_base = 0.0f;
       } else {
-        mx = fmaf(row_max128(s), sl, rowb2);
+        mx = fmaf(s_int ? (float)row_max128_s32(s) : row_max128(s), sl, rowb2);
         scl = sl;
         off_base = rowb2;
       }
@@ -442,7 +457,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float off = off_base - m_use;
       // columns in pairs: one packed FMA forms both exponents, one packed add accumulates
       // both probabilities (two accumulators break the dependency chain)
-      const uint64_t scl2 = f32x2_pack(scl, scl), off2 = f32x2_pack(off, off);
+      // integer S: x = (S + 1.5 * 2^23) * scl + (off - 1.5 * 2^23 * scl), the addend in one rounding
+      const uint32_t s_add = s_int ? 0x4B400000u : 0u;
+      const float off_x = s_int ? fmaf(-12582912.0f, scl, off) : off;
+      const uint64_t scl2 = f32x2_pack(scl, scl), off2 = f32x2_pack(off_x, off_x);
       uint64_t lsum2[2] = {0ull, 0ull};
 #pragma unroll
       for (int qtr = 0; qtr < 4; ++qtr) {
@@ -453,7 +471,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int c2 = 0; c2 < 32; c2 += 2) {
           const int c = qtr * 32 + c2;
           float x0, x1;
-          f32x2_unpack(f32x2_fma(f32x2_pack_bits(s[c], s[c + 1]), scl2, off2), x0, x1);
+          f32x2_unpack(f32x2_fma(f32x2_pack_bits(s[c] + s_add, s[c + 1] + s_add), scl2, off2), x0, x1);
           const float p0 = ex2_approx(x0);
           const float p1 = ex2_approx(x1);
           lsum2[(c >> 1) & 1] = f32x2_add(lsum2[(c >> 1) & 1], f32x2_pack(p0, p1));
