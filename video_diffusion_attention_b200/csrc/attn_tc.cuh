@@ -377,6 +377,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       float rowb2 = 0.0f;
       if (is_tgt) {
         if (cls == kClsConstCap) rowb2 = cval * kLog2e;
+        else if (cls == kClsRowGuide) rowb2 = -penalty_f32(fabsf(t_q - kr.tk_min), bp) * kLog2e;
         else if (cls == kClsConstPic)
           rowb2 = (bp.n_extra > 0 ? m_q * cval + wx[kr.single_pic & 15] : m_q * cval) * kLog2e;
       }

@@ -53,6 +53,7 @@ constexpr int kClsZero = 0;      // no edge of the pair is biased
 constexpr int kClsConstCap = 1;  // every target-row x key edge carries exactly -cap
 constexpr int kClsConstPic = 2;  // every target-row x key edge carries m_row * ln(gain_p)
 constexpr int kClsFull = 3;      // evaluate the bias edge by edge
+constexpr int kClsRowGuide = 4;  // every valid key is GUIDE at one time: -penalty per target row
 
 // The temporal penalty in fp32: min(strength * (max(dt - window, 0) / falloff)^2, cap)
 // ("TARA: Native Temporal Alignment for MiniMax H3 References", "The temporal rule").
@@ -84,6 +85,8 @@ __device__ __forceinline__ int classify_pair(const TileRec& q, const TileRec& k,
         *cval = -p.cap;
         return kClsConstCap;
       }
+      // a key tile inside one guide frame: the bias depends on the query row only
+      if (k.tk_min == k.tk_max) return kClsRowGuide;
     }
     return kClsFull;
   }
