@@ -131,6 +131,25 @@ def test_parameter_corners(p):
     _check(_small("par", "bf16", 128, _layout(tpf=50, frames=8), p, H=2))
 
 
+@pytest.mark.parametrize("p", [
+    W.Params(),
+    W.Params(window=0.0, falloff=0.05, strength=5.0, cap=12.0),
+    W.Params(window=0.3, falloff=1.0, strength=0.5, cap=2.0, gain=(1.5,) + (1.0,) * 8),
+])
+def test_single_frame_guide_tiles(p):
+    # guide frames of exactly one 128-token tile: every near-diagonal guide key tile holds one
+    # time, so the per-row guide class carries the temporal bias; the offset target start puts
+    # query tiles across two target frames
+    segs = [
+        W.Segment(W.TEXT, 1, 128),
+        W.Segment(W.PICTURE, 1, 128, pic=1),
+        W.Segment(W.GUIDE, 9, 128, frame_dt_s=4 / 24),
+        W.Segment(W.TARGET, 9, 128, t0_s=1 / 24, frame_dt_s=4 / 24, mask=W.uniform_mask(5, 128)),
+        W.Segment(W.AUDIO, 1, 77),
+    ]
+    _check(_small("sfg", "bf16", 128, segs, p, H=2, qk=1.5, seed=410))
+
+
 def test_unsorted_roles_and_other_video():
     # roles interleaved out of the usual order, plus a non-selected video reference
     segs = [
