@@ -165,6 +165,30 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
                       const tara_token_meta* meta, const tara_params* p,
                       tara_tensor* O, float* LSE, void* stream);
 
+/* ---- host buffers ------------------------------------------------------------------------ */
+/* The same operation with Q, K, V, O, LSE and every metadata array (seg, time_s, pic, m,
+ * extra_m) in HOST memory; pinned memory (cudaHostAlloc / cudaHostRegister) lets the copies
+ * overlap the kernels, pageable memory works but serialises them.  The pages have no
+ * counterpart: it is the runtime around the kernel for callers whose tensors live on the host.
+ *   The B*H (branch, head) planes are processed in chunks of consecutive planes (about 1 GiB of
+ *   Q, K, V and O each, within one branch when the metadata is per branch): per chunk, the
+ *   host->device copies of Q, K, V run on one internal stream, the attention
+ *   (tara_attn_forward on device chunk buffers) on a second, and the device->host copies of O
+ *   and LSE on a third, with two chunk buffer sets alternating, so transfers overlap kernels.
+ *   Ordering: everything runs after the work already queued on `stream`, and `stream` waits
+ *   for the last copy; the call itself does not block the host.  The host buffers must stay
+ *   valid and unmodified until `stream` has completed (as with cudaMemcpyAsync).
+ *   Device memory: the metadata plus two chunk sets, cached per device and grown with
+ *   cudaMalloc (a growth synchronises the device).  A kernel-event pair pending for the
+ *   calling thread (tara_set_kernel_events) is dropped.
+ * Same arguments and checks as tara_attn_forward (shapes, dtypes, parameters, extra
+ * bindings) except that pointers are host pointers with no alignment requirement.
+ * Errors: TARA_ERR_NULL, _SHAPE, _DTYPE, _HEAD_DIM, _PARAM, _ALIGN, _TOO_LARGE, TARA_ERR_CUDA;
+ * an error after the first copy was queued still leaves `stream` waiting for the queued work. */
+int tara_attn_forward_host(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
+                           const tara_token_meta* meta, const tara_params* p,
+                           tara_tensor* O, float* LSE, void* stream);
+
 /* ---- 8-bit quantisation of Q and K ------------------------------------------------------ */
 /* The quantisation tara_attn_forward runs when p->qk_int8 = 1, exposed for callers that keep
  * the codes ("TARA: ...", "Three backends" names dense INT8 kernels without their scaling;

@@ -218,6 +218,32 @@ def test_quantize_argument_checks(lib):
     assert _quant_call(lib, K=_t(ptr=FAKE + 4)) == -6
 
 
+def test_host_forward_argument_checks(lib):
+    def call(Q=None, K=None, V=None, meta=None, p=None, O=None, lse=FAKE):
+        Q, K, V, O = (x if x is not None else _t() for x in (Q, K, V, O))
+        meta = meta if meta is not None else _meta()
+        p = p if p is not None else B.make_params()
+        return lib.tara_attn_forward_host(ctypes.byref(Q), ctypes.byref(K), ctypes.byref(V),
+                                          ctypes.byref(meta), ctypes.byref(p), ctypes.byref(O),
+                                          ctypes.c_void_p(lse), None)
+    assert lib.tara_attn_forward_host(None, None, None, None, None, None, None, None) == -1
+    assert call(lse=0) == -1
+    assert call(meta=_meta(ptr=0)) == -1
+    assert call(K=_t(dtype=B.TARA_FP16)) == -3
+    assert call(V=_t(shape=(1, 2, 301, 128))) == -2
+    assert call(meta=_meta(N=301)) == -2
+    s96 = (1, 2, 300, 96)
+    assert call(Q=_t(shape=s96), K=_t(shape=s96), V=_t(shape=s96), O=_t(shape=s96)) == -4
+    assert call(p=B.make_params(falloff=0.0)) == -5
+    assert call(p=B.make_params(qk_int8=3)) == -5
+    f = B.TARA_FP32
+    assert call(Q=_t(dtype=f), K=_t(dtype=f), V=_t(dtype=f), O=_t(dtype=f),
+                p=B.make_params(qk_int8=1)) == -3
+    p1 = B.make_params(extra_gain=((1.5,) * 9,))
+    assert call(p=p1, meta=_meta(extra=None, extra_stride=300)) == -1
+    assert call(p=p1, meta=_meta(extra=FAKE, extra_stride=10)) == -2
+
+
 # ---------------------------------------------------------------------------------------
 # the packer against the oracle's packer (bit-exact) and its error handling
 # ---------------------------------------------------------------------------------------

@@ -12,7 +12,7 @@ All compute runs in libtara_attn.so (C ABI in include/tara_attn.h); this package
 marshals arguments.  Build the library with `python -m video_diffusion_attention_b200.build`.
 """
 from ._binding import (  # noqa: F401
-    DeviceMeta, TaraError, attn_forward, default_params, device_status, load_library,
+    DeviceMeta, HostMeta, TaraError, attn_forward, attn_forward_host, default_params, device_status, load_library,
     make_params, pack_token_meta, packed_length, params_from, prepare_target_mask,
     quantize_qk_int8, selftest_wait, set_kernel_events, SEG_AUDIO, SEG_GUIDE,
     SEG_OTHER_VIDEO, SEG_PICTURE, SEG_TARGET, SEG_TEXT, TARA_BF16, TARA_FP16, TARA_FP32,

@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = ("tara_default_params", "tara_status_string", "tara_attn_forward",
            "tara_device_status", "tara_packed_length", "tara_pack_token_meta",
            "tara_set_kernel_events", "tara_selftest_wait", "tara_attn_forward_noalloc",
-           "tara_prepare_target_mask", "tara_quantize_qk_int8")
+           "tara_prepare_target_mask", "tara_quantize_qk_int8", "tara_attn_forward_host")
 
 
 class TaraError(RuntimeError):
@@ -90,6 +90,8 @@ def load_library(path: Optional[str] = None):
         ctypes.c_void_p, ctypes.c_void_p]
     lib.tara_attn_forward_noalloc.restype = ctypes.c_int
     lib.tara_attn_forward_noalloc.argtypes = lib.tara_attn_forward.argtypes
+    lib.tara_attn_forward_host.restype = ctypes.c_int
+    lib.tara_attn_forward_host.argtypes = lib.tara_attn_forward.argtypes
     lib.tara_quantize_qk_int8.restype = ctypes.c_int
     lib.tara_quantize_qk_int8.argtypes = [ctypes.POINTER(TaraTensor)] * 2 + [ctypes.c_void_p] * 5
     lib.tara_set_kernel_events.restype = ctypes.c_int
@@ -230,6 +232,27 @@ class DeviceMeta:
         return c
 
 
+class HostMeta(DeviceMeta):
+    """Per-token metadata in (pinned) host memory, for attn_forward_host."""
+
+    def __init__(self, meta: dict, batch_stride: int = 0, N: Optional[int] = None,
+                 pin: bool = True):
+        import torch
+        def host(a, dt):
+            t = torch.as_tensor(np.ascontiguousarray(a), dtype=dt).contiguous()
+            return t.pin_memory() if pin else t
+        self.seg = host(meta["seg"], torch.uint8)
+        self.time_s = host(meta["time_s"], torch.float32)
+        self.pic = host(meta["pic"], torch.uint8)
+        self.m = host(meta["m"], torch.float32)
+        self.extra_m = None
+        if meta.get("m_extra") is not None and len(meta["m_extra"]) > 0:
+            self.extra_m = host(np.asarray(meta["m_extra"], np.float32).reshape(
+                -1, self.m.numel()), torch.float32)
+        self.batch_stride = int(batch_stride)
+        self.N = int(self.seg.numel()) if N is None else int(N)
+
+
 def _dtype_code(t) -> int:
     import torch
     return {torch.bfloat16: TARA_BF16, torch.float16: TARA_FP16, torch.float32: TARA_FP32}[t.dtype]
@@ -264,6 +287,36 @@ def attn_forward(q, k, v, meta: DeviceMeta, params: TaraParams, out=None, lse=No
                                ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
     if rc != 0:
         raise TaraError(rc, "tara_attn_forward")
+    return out, lse
+
+
+def attn_forward_host(q, k, v, meta: "HostMeta", params: TaraParams, out=None, lse=None,
+                      stream=None):
+    """The forward on host tensors ([B][H][N][D] CPU tensors, pinned for overlap): copies,
+    kernels and copies back run as a chunked three-stream pipeline inside the library.
+
+    Asynchronous on `stream` (default: the current CUDA stream); synchronise it before reading
+    `out` / `lse` or touching the inputs."""
+    import torch
+    lib = load_library()
+    B, H, N, D = q.shape
+    if out is None:
+        out = torch.empty_like(q, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    for t in (q, k, v, out, lse):
+        if t.is_cuda:
+            raise ValueError("attn_forward_host takes host tensors")
+    cq, ck, cv, co = tensor_struct(q), tensor_struct(k), tensor_struct(v), tensor_struct(out)
+    cm = meta.c_struct()
+    rc = lib.tara_attn_forward_host(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv),
+                                    ctypes.byref(cm), ctypes.byref(params), ctypes.byref(co),
+                                    ctypes.c_void_p(lse.data_ptr()),
+                                    ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise TaraError(rc, "tara_attn_forward_host")
     return out, lse
 
 

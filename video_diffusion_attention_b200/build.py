@@ -13,7 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libtara_attn.so")
-SOURCES = [os.path.join(CSRC, "tara_abi.cu"), os.path.join(CSRC, "tara_pack.cpp")]
+SOURCES = [os.path.join(CSRC, "tara_abi.cu"), os.path.join(CSRC, "tara_pack.cpp"),
+           os.path.join(CSRC, "tara_host.cpp")]
 HEADERS = [os.path.join(ROOT, "include", "tara_attn.h")] + [
     os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cuh", ".h"))]
 

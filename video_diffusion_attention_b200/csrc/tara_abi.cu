@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "tara_attn.h"
+#include "param_checks.h"
 #include "attn_simt.cuh"
 #include "attn_pair.cuh"
 #include "attn_tc.cuh"
@@ -76,26 +77,7 @@ int get_encode_fn() {
   return TARA_OK;
 }
 
-bool finite_f(float x) { return std::isfinite(x); }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-int check_params(const tara_params* p) {
-  if (!finite_f(p->window) || !finite_f(p->falloff) || !finite_f(p->strength) ||
-      !finite_f(p->cap) || !finite_f(p->softmax_scale))
-    return TARA_ERR_PARAM;
-  if (p->falloff <= 0.0f || p->window < 0.0f || p->strength < 0.0f || p->cap < 0.0f ||
-      p->softmax_scale < 0.0f)
-    return TARA_ERR_PARAM;
-  for (int i = 0; i < 9; ++i)
-    if (!finite_f(p->gain[i]) || p->gain[i] <= 0.0f) return TARA_ERR_PARAM;
-  if (p->n_extra_bindings < 0 || p->n_extra_bindings > TARA_MAX_EXTRA_BINDINGS)
-    return TARA_ERR_PARAM;
-  for (int k = 0; k < p->n_extra_bindings; ++k)
-    for (int i = 0; i < 9; ++i)
-      if (!finite_f(p->extra_gain[k][i]) || p->extra_gain[k][i] <= 0.0f) return TARA_ERR_PARAM;
-  if (p->qk_int8 != 0 && p->qk_int8 != 1) return TARA_ERR_PARAM;
-  return TARA_OK;
-}
 
 BiasParams make_bias_params(const tara_params* p, int D) {
   BiasParams bp;
