@@ -61,9 +61,13 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+# the device sources the attention kernel is compiled from
+KERNEL_SOURCES = ("attn_tc.cuh", "sm100_ptx.cuh", "tara_common.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
+    for f in KERNEL_SOURCES:
         with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
