@@ -366,7 +366,7 @@ def main():
         torch.cuda.synchronize(dev)
         mms = m0.elapsed_time(m1) / reps
         mbytes = px.numel() * 4 + mo.numel() * 4
-        mask_line = {"kernel": "target_mask_kernel", "workload": "107x544x928 fp32 pixel mask -> "
+        mask_line = {"kernel": "target_mask_narrow_kernel (rows <= 1024 px)", "workload": "107x544x928 fp32 pixel mask -> "
                      "%dx40x50 target weights" % tgt[0].frames, "ms": mms, "bound": "hbm",
                      "algorithmic_bytes": mbytes, "achieved_GBs": mbytes / (mms * 1e-3) / 1e9}
     # the INT8 Q K^T variant of the same forward (Q per token, K per 128-key block, 8-bit

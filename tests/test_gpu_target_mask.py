@@ -18,6 +18,9 @@ CASES = [
     (5, 7, 10, 5, 1, 5, 3, 4),               # tiny, one pixel frame per latent frame
     (39, 20, 24, 39, 4, 10, 40, 50),         # upsampling (patch grid finer than the mask)
     (107, 720, 1280, 107, 4, 27, 40, 50),    # pixel-resolution mask of the full shot
+    (107, 544, 928, 107, 4, 27, 40, 50),     # the pages' user-run resolution (narrow rows)
+    (22, 33, 1024, 22, 4, 6, 7, 50),         # widest narrow-row case
+    (22, 33, 1028, 22, 4, 6, 7, 50),         # just past it: the general kernel
 ]
 
 

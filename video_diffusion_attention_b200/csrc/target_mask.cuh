@@ -105,4 +105,66 @@ target_mask_kernel(const float* __restrict__ mask, int F_in, int Hp, int Wp, int
   }
 }
 
+// Narrow rows (Wp <= 1024, every pixel row 16-byte aligned): thread t owns columns 4t..4t+3,
+// one 16-byte load per pixel row, and walks the (pixel frame, pixel row) pairs of its cell
+// row eight at a time so that eight loads are in flight per thread.
+__global__ void __launch_bounds__(kMaskThreads)
+target_mask_narrow_kernel(const float* __restrict__ mask, int F_in, int Hp, int Wp, int L,
+                          int tau, int F_lat, int Hq, int Wq, float* __restrict__ out) {
+  extern __shared__ float cell_acc[];   // [Wq]
+  const int y = blockIdx.x;
+  const int f = blockIdx.y;
+  const int tid = threadIdx.x;
+  for (int x = tid; x < Wq; x += kMaskThreads) cell_acc[x] = 0.0f;
+  __syncthreads();
+
+  const long long ylo = (long long)y * Hp, yhi = (long long)(y + 1) * Hp;
+  const int r0 = (int)(ylo / Hq);
+  const int r1 = (int)((yhi + Hq - 1) / Hq);
+  int t0 = 0, t1 = 1;
+  if (F_in > 1) {
+    t0 = f * tau;
+    t1 = min(t0 + tau, L);
+  }
+  const int nr = r1 - r0;
+  const int npairs = (t1 - t0) * nr;
+  const int c = tid * 4;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (c < Wp) {
+#pragma unroll 8
+    for (int i = 0; i < npairs; ++i) {
+      const int t = t0 + i / nr;
+      const int r = r0 + i % nr;
+      const long long rlo = (long long)r * Hq;
+      const float wy = (float)(min(yhi, rlo + Hq) - max(ylo, rlo));
+      const float4 v = __ldg(reinterpret_cast<const float4*>(mask + ((long long)t * Hp + r) * Wp + c));
+      acc.x = fmaf(wy, v.x, acc.x);
+      acc.y = fmaf(wy, v.y, acc.y);
+      acc.z = fmaf(wy, v.z, acc.z);
+      acc.w = fmaf(wy, v.w, acc.w);
+    }
+    const float cs[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const long long clo = (long long)(c + k) * Wq, chi = clo + Wq;
+      for (int x = (int)(clo / Wp); x < Wq && (long long)x * Wp < chi; ++x) {
+        const long long xlo = (long long)x * Wp;
+        const float wx = (float)(min(xlo + Wp, chi) - max(xlo, clo));
+        atomicAdd(&cell_acc[x], wx * cs[k]);
+      }
+    }
+  }
+  __syncthreads();
+
+  const float norm = 1.0f / ((float)Hp * (float)Wp * (float)(t1 - t0));
+  for (int x = tid; x < Wq; x += kMaskThreads) {
+    const float v = cell_acc[x] * norm;
+    if (F_in > 1) {
+      out[((long long)f * Hq + y) * Wq + x] = v;
+    } else {
+      for (int ff = 0; ff < F_lat; ++ff) out[((long long)ff * Hq + y) * Wq + x] = v;
+    }
+  }
+}
+
 }  // namespace tara
