@@ -11,7 +11,6 @@
 #include "tara_attn.h"
 #include "param_checks.h"
 #include "attn_simt.cuh"
-#include "attn_pair.cuh"
 #include "attn_tc.cuh"
 #include "quant_int8.cuh"
 #include "target_mask.cuh"
@@ -25,20 +24,12 @@ __device__ int g_device_status;
 
 constexpr int kMaxDevices = 64;
 
-// 1: head dim 128 runs on the SM-pair kernel (attn_pair.cuh, 2-SM MMA, S double-buffered;
-// parity-tested, measured slower here: the pair handoff latency outweighs the overlap);
-// 0 (default): on the single-SM kernel (attn_tc.cuh).
-#ifndef TARA_PAIR_KERNEL
-#define TARA_PAIR_KERNEL 0
-#endif
-
 struct DeviceState {
   void* ws = nullptr;           // tile summaries + per-key records
   size_t ws_bytes = 0;
   int* status = nullptr;        // device address of g_device_status
   bool tc_attr_set[2][2] = {{false, false}, {false, false}};   // [bf16][D==128]
   bool tc_q8_attr_set[2] = {false, false};                     // [bf16], D = 128
-  bool pair_attr_set[2] = {false, false};                      // [bf16]
   bool simt_attr_set = false;
 };
 
@@ -104,13 +95,13 @@ BiasParams make_bias_params(const tara_params* p, int D) {
   return bp;
 }
 
-int encode_qkv_map(CUtensorMap* map, const tara_tensor* t, uint32_t box_rows = kTile) {
+int encode_qkv_map(CUtensorMap* map, const tara_tensor* t) {
   const CUtensorMapDataType dt =
       t->dtype == TARA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const cuuint64_t dims[3] = {(cuuint64_t)t->D, (cuuint64_t)t->N,
                               (cuuint64_t)t->B * (cuuint64_t)t->H};
   const cuuint64_t strides[2] = {(cuuint64_t)t->D * 2, (cuuint64_t)t->N * (cuuint64_t)t->D * 2};
-  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, dt, 3, t->ptr, dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -234,28 +225,6 @@ int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& m
   dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
   if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
   attn_tc_kernel<kBF16, D, kQ8><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, a);
-  if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
-  return record_stop(stream);
-}
-
-// D = 128: the SM-pair kernel (two CTAs per 256 query rows, K tiles loaded as 64-row halves).
-template <bool kBF16>
-int launch_pair(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V, const TcArgs& a,
-                int B, int H, int ntiles, cudaStream_t stream, bool* attr) {
-  constexpr int smem = PairShape::kSmemBytes;
-  if (!*attr) {
-    if (cudaFuncSetAttribute(attn_pair_kernel<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return TARA_ERR_CUDA;
-    *attr = true;
-  }
-  CUtensorMap mq, mk, mv;
-  if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K, 64) != TARA_OK ||
-      encode_qkv_map(&mv, V) != TARA_OK)
-    return TARA_ERR_CUDA;
-  dim3 grid((unsigned)((ntiles + 1) / 2 * 2), (unsigned)H, (unsigned)B);
-  if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
-  attn_pair_kernel<kBF16><<<grid, 384, smem, stream>>>(mq, mk, mv, a);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
   return record_stop(stream);
 }
@@ -438,15 +407,9 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
   if (q8)
     return bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
                 : launch_tc<false, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st);
-#if TARA_PAIR_KERNEL
-  if (D == 128)
-    return bf16 ? launch_pair<true>(Q, K, V, a, B, H, ntiles, stream, &st->pair_attr_set[1])
-                : launch_pair<false>(Q, K, V, a, B, H, ntiles, stream, &st->pair_attr_set[0]);
-#else
   if (D == 128)
     return bf16 ? launch_tc<true, 128>(mq, mk, mv, a, B, H, ntiles, stream, st)
                 : launch_tc<false, 128>(mq, mk, mv, a, B, H, ntiles, stream, st);
-#endif
   return bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
               : launch_tc<false, 64>(mq, mk, mv, a, B, H, ntiles, stream, st);
 }
@@ -649,17 +612,9 @@ extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor
   a.q_scale = nullptr;
   a.k_scale = nullptr;
   const bool bf16 = Q->dtype == TARA_BF16;
-#if TARA_PAIR_KERNEL
-  if (D == 128) {
-    bool attr = false;
-    return bf16 ? launch_pair<true>(Q, K, V, a, B, H, ntiles, stream, &attr)
-                : launch_pair<false>(Q, K, V, a, B, H, ntiles, stream, &attr);
-  }
-#else
   if (D == 128)
     return bf16 ? launch_tc_static<true, 128>(mq, mk, mv, a, B, H, ntiles, stream)
                 : launch_tc_static<false, 128>(mq, mk, mv, a, B, H, ntiles, stream);
-#endif
   return bf16 ? launch_tc_static<true, 64>(mq, mk, mv, a, B, H, ntiles, stream)
               : launch_tc_static<false, 64>(mq, mk, mv, a, B, H, ntiles, stream);
 }
