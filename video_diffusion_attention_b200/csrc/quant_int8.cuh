@@ -33,45 +33,61 @@ __device__ __forceinline__ uint32_t q8_code(float x, float inv, bool live) {
   return (uint32_t)(c & 0xFF);
 }
 
-// Q: one warp per token row of D (64 or 128) values; lane l owns values 4l..4l+3 (D=128) or
-// 2l..2l+1 (D=64).  rows = B*H*N.
+// Q: rows of D (64 or 128) values, 16 bytes (8 values) per lane, so D/8 lanes per row and
+// 32/(D/8) rows per warp-wide load; each warp walks kQRowsUnroll such row groups at once, so
+// that many 16-byte loads are in flight per lane.  The row amax is a max over the row's lanes
+// (shuffles within the lane group).  rows = B*H*N.
+constexpr int kQRowsUnroll = 4;
+
 template <bool kBF16, int D>
 __global__ void __launch_bounds__(kQ8Threads)
 quant_q_kernel(const uint16_t* __restrict__ x, long long rows, int8_t* __restrict__ codes,
                float* __restrict__ scales) {
-  constexpr int kPer = D / 32;
-  const long long row = (long long)blockIdx.x * (kQ8Threads / 32) + (threadIdx.x >> 5);
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerLoad = 32 / kLanesPerRow;
+  constexpr int kRowsPerWarp = kRowsPerLoad * kQRowsUnroll;
   const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const uint16_t* src = x + row * D + lane * kPer;
-  float v[kPer];
-  if (kPer == 4) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(src);
-    v[0] = widen16<kBF16>((uint16_t)(raw.x & 0xFFFFu));
-    v[1] = widen16<kBF16>((uint16_t)(raw.x >> 16));
-    v[2] = widen16<kBF16>((uint16_t)(raw.y & 0xFFFFu));
-    v[3] = widen16<kBF16>((uint16_t)(raw.y >> 16));
-  } else {
-    const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
-    v[0] = widen16<kBF16>((uint16_t)(raw & 0xFFFFu));
-    v[1] = widen16<kBF16>((uint16_t)(raw >> 16));
+  const int sub = lane % kLanesPerRow;          // this lane's 8 values within the row
+  const int grp = lane / kLanesPerRow;          // which row of a load group
+  const long long warp_row0 =
+      ((long long)blockIdx.x * (kQ8Threads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp;
+  uint4 raw[kQRowsUnroll];
+#pragma unroll
+  for (int u = 0; u < kQRowsUnroll; ++u) {
+    const long long row = warp_row0 + u * kRowsPerLoad + grp;
+    raw[u] = row < rows ? *reinterpret_cast<const uint4*>(x + row * D + sub * 8)
+                        : make_uint4(0u, 0u, 0u, 0u);
   }
-  // |x| as bits: non-negative floats order like unsigned integers
-  uint32_t am = 0;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) am = max(am, __float_as_uint(v[i]) & 0x7FFFFFFFu);
-  am = __reduce_max_sync(0xffffffffu, am);
-  const float amax = __uint_as_float(am);
-  const bool live = amax > kQ8AmaxFloor;
-  const float inv = live ? __fdiv_rn(kQ8Max, amax) : 0.0f;
-  uint32_t packed = 0;
+  for (int u = 0; u < kQRowsUnroll; ++u) {
+    const long long row = warp_row0 + u * kRowsPerLoad + grp;
+    const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+    float v[8];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) packed |= q8_code(v[i], inv, live) << (8 * i);
-  if (kPer == 4)
-    *reinterpret_cast<uint32_t*>(codes + row * D + lane * kPer) = packed;
-  else
-    *reinterpret_cast<uint16_t*>(codes + row * D + lane * kPer) = (uint16_t)packed;
-  if (lane == 0) scales[row] = live ? __fdiv_rn(amax, kQ8Max) : 0.0f;
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = widen16<kBF16>((uint16_t)(w[k] & 0xFFFFu));
+      v[2 * k + 1] = widen16<kBF16>((uint16_t)(w[k] >> 16));
+    }
+    // |x| as bits: non-negative floats order like unsigned integers
+    uint32_t am = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) am = max(am, __float_as_uint(v[k]) & 0x7FFFFFFFu);
+#pragma unroll
+    for (int o = kLanesPerRow / 2; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+    const float amax = __uint_as_float(am);
+    const bool live = amax > kQ8AmaxFloor;
+    const float inv = live ? __fdiv_rn(kQ8Max, amax) : 0.0f;
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      lo |= q8_code(v[k], inv, live) << (8 * k);
+      hi |= q8_code(v[4 + k], inv, live) << (8 * k);
+    }
+    if (row < rows) {
+      *reinterpret_cast<uint2*>(codes + row * D + sub * 8) = make_uint2(lo, hi);
+      if (sub == 0) scales[row] = live ? __fdiv_rn(amax, kQ8Max) : 0.0f;
+    }
+  }
 }
 
 // K: one CTA per (branch x head, 128-token block).  The block is contiguous in [N][D] memory;

@@ -138,7 +138,9 @@ int launch_quant(const tara_tensor* Q, const tara_tensor* K, int8_t* qc, float* 
   const bool bf16 = Q->dtype == TARA_BF16;
   const int BH = Q->B * Q->H, N = Q->N, D = Q->D;
   const long long rows = (long long)BH * N;
-  const unsigned qgrid = (unsigned)((rows + (kQ8Threads / 32) - 1) / (kQ8Threads / 32));
+  // rows per CTA: its warps x (32 / (D/8)) rows per load x kQRowsUnroll loads
+  const long long q_rows_cta = (long long)(kQ8Threads / 32) * (256 / D) * kQRowsUnroll;
+  const unsigned qgrid = (unsigned)((rows + q_rows_cta - 1) / q_rows_cta);
   const dim3 kgrid((unsigned)((N + kQ8Block - 1) / kQ8Block), (unsigned)BH);
   const int nb = (N + kQ8Block - 1) / kQ8Block;
   const uint16_t* q = static_cast<const uint16_t*>(Q->ptr);
