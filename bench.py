@@ -180,6 +180,19 @@ def oracle_sample_rate(w: W.Workload, budget_s: float, device_inputs=None, seed:
     return n, dt, threads
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def run_reference(args, w: W.Workload):
     """The oracle arm: K timed steps, each a bounded row sample of the workload."""
     import oracle
@@ -217,7 +230,7 @@ def run_reference(args, w: W.Workload):
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": describe(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "cpu_model": cpu_model(), "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -314,6 +327,7 @@ def main():
         raise SystemExit("kernel reported a device timeout in the timed region")
     ms_total = start.elapsed_time(stop)
     kernel_ms = [a.elapsed_time(b) for a, b in kev]
+    kernel_ms_median = statistics.median(kernel_ms)
     ms_total, kmean = max_over_ranks([ms_total, statistics.mean(kernel_ms)], dev)
     ms_step = ms_total / args.steps
     value = job_throughput(w.flops, world, ms_step)
@@ -427,6 +441,7 @@ def main():
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "attn_tc_kernel", "kernel_ms": kmean,
+                     "kernel_ms_median": kernel_ms_median,
                      "peak_kind": "bf16_tflops_sustained (%s): the kernel runs back to back for "
                                   "seconds" % peak_src},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
@@ -442,9 +457,10 @@ def main():
         n, dt, threads = oracle_sample_rate(w, args.cpu_budget, device_inputs=(q, k, v))
         line["cpu_baseline"] = {
             "value": n * 4.0 * w.N * w.D / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(),
             "sample": "%d seeded query rows of %s in %.1f s (each row against all %d keys, "
-                      "fp64)" % (n, w.name, dt, w.N)}
+                      "fp64)" % (n, w.name, dt, w.N),
+            "extrapolated_full_call_s": dt / n * w.B * w.H * w.N}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
