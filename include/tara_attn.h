@@ -32,13 +32,16 @@
  *     entry point exits, throws or prints.
  *   - Ownership: the caller owns every buffer.  Device buffers are never freed or retained by
  *     the library beyond the call.  tara_attn_forward keeps one internal per-device workspace
- *     (tile summaries and per-key bias records, about 8 bytes per token plus 32 bytes per
- *     128-token tile per metadata set); it is allocated with cudaMalloc the first time a
- *     device sees a given size and reused afterwards, so the first call on a device (or with a
- *     larger N) must not be made while a stream is being captured.
+ *     (per metadata set 16 bytes per token plus 32 bytes per 128-token tile; with qk_int8,
+ *     also 2*B*H*N*D bytes of codes and 4*B*H*(N + N/128) bytes of scales); it is allocated
+ *     with cudaMalloc the first time a device sees a given size and reused afterwards, so the
+ *     first call on a device (or with a larger size) must not be made while a stream is being
+ *     captured.
  *   - Asynchrony: device work is enqueued on `stream` and the call returns without
- *     synchronising.  Calls on different streams that use the same device share the
- *     workspace and therefore must not overlap; serialise them on one stream.
+ *     synchronising.  Calls on different streams of one device share the workspace: each
+ *     16-bit call makes its stream wait (an event) for the previous call's kernels before
+ *     rewriting it, so such calls run one after the other on the GPU.  Calls made while their
+ *     stream is being captured skip that ordering; serialise captured work on one stream.
  */
 #ifndef TARA_ATTN_H_
 #define TARA_ATTN_H_

@@ -167,3 +167,31 @@ def test_batch_of_branches_shared_and_strided_meta():
     w = _small("br", "bf16", 128, _layout(tpf=40, frames=4), GAINS, H=2, B=3)
     _check(w)
     _check(w, per_branch_meta=True)
+
+
+def test_calls_on_two_streams_do_not_share_summaries_concurrently():
+    # two shots of the same length with different role layouts, launched back to back on two
+    # streams: the library orders them on the shared workspace, so each matches its own
+    # single-stream result bit for bit
+    import video_diffusion_attention_b200 as T
+    segs_a = _layout(tpf=64, frames=6)
+    segs_b = [W.Segment(W.TEXT, 1, 37), W.Segment(W.PICTURE, 1, 96, pic=2),
+              W.Segment(W.GUIDE, 6, 64, t0_s=0.3, frame_dt_s=4 / 24),
+              W.Segment(W.TARGET, 6, 64, frame_dt_s=4 / 24), W.Segment(W.AUDIO, 1, 21)]
+    wa = _small("sa", "bf16", 128, segs_a, GAINS, H=8, seed=600)
+    wb = _small("sb", "bf16", 128, segs_b, GAINS, H=8, seed=601)
+    assert wa.N == wb.N
+    ins = [tuple(t.to(DEV) for t in W.make_qkv(w, DEV)) for w in (wa, wb)]
+    metas = [T.DeviceMeta(T.pack_token_meta(w.segments), DEV) for w in (wa, wb)]
+    params = [T.params_from(w.params) for w in (wa, wb)]
+    ref = [T.attn_forward(*ins[i], metas[i], params[i]) for i in range(2)]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for _ in range(3):
+        for i in range(2):
+            outs.append((i, T.attn_forward(*ins[i], metas[i], params[i], stream=streams[i])))
+    torch.cuda.synchronize()
+    assert T.device_status() == 0
+    for i, (O, L) in outs:
+        assert torch.equal(O, ref[i][0]) and torch.equal(L, ref[i][1])

@@ -31,6 +31,9 @@ struct DeviceState {
   bool tc_attr_set[2][2] = {{false, false}, {false, false}};   // [bf16][D==128]
   bool tc_q8_attr_set[2] = {false, false};                     // [bf16], D = 128
   bool simt_attr_set = false;
+  // recorded on a call's stream after its last workspace reader; the next call's stream waits
+  // on it before rewriting the workspace, so calls on different streams serialise on the GPU
+  cudaEvent_t ws_free = nullptr;
 };
 
 std::mutex g_mu;
@@ -371,6 +374,17 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
   float* qs = reinterpret_cast<float*>(ws + rec_bytes + key_bytes + 2 * code_bytes);
   float* ks = reinterpret_cast<float*>(ws + rec_bytes + key_bytes + 2 * code_bytes + qs_bytes);
 
+  // wait for the previous call's kernels to finish reading the workspace (not while the stream
+  // is being captured: a captured wait on an event recorded outside the graph is not allowed)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return TARA_ERR_CUDA;
+  const bool order_ws = cap == cudaStreamCaptureStatusNone;
+  if (order_ws) {
+    if (!st->ws_free && cudaEventCreateWithFlags(&st->ws_free, cudaEventDisableTiming) != cudaSuccess)
+      return TARA_ERR_CUDA;
+    if (cudaStreamWaitEvent(stream, st->ws_free, 0) != cudaSuccess) return TARA_ERR_CUDA;
+  }
+
   CUtensorMap mq, mk, mv;
   if (q8) {
     if (encode_q8_map(&mq, qc, B * H, N, D) != TARA_OK ||
@@ -407,13 +421,17 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
   a.k_scale = ks;
   const bool bf16 = Q->dtype == TARA_BF16;
   if (q8)
-    return bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
-                : launch_tc<false, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st);
-  if (D == 128)
-    return bf16 ? launch_tc<true, 128>(mq, mk, mv, a, B, H, ntiles, stream, st)
-                : launch_tc<false, 128>(mq, mk, mv, a, B, H, ntiles, stream, st);
-  return bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
+    rc = bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
+              : launch_tc<false, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st);
+  else if (D == 128)
+    rc = bf16 ? launch_tc<true, 128>(mq, mk, mv, a, B, H, ntiles, stream, st)
+              : launch_tc<false, 128>(mq, mk, mv, a, B, H, ntiles, stream, st);
+  else
+    rc = bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
               : launch_tc<false, 64>(mq, mk, mv, a, B, H, ntiles, stream, st);
+  if (rc == TARA_OK && order_ws && cudaEventRecord(st->ws_free, stream) != cudaSuccess)
+    return TARA_ERR_CUDA;
+  return rc;
 }
 
 int tara_quantize_qk_int8(const tara_tensor* Q, const tara_tensor* K, int8_t* q_codes,
