@@ -160,9 +160,20 @@ extern "C" int tara_attn_forward_host(const tara_tensor* Q, const tara_tensor* K
   char* ho = static_cast<char*>(O->ptr);
   char* hl = reinterpret_cast<char*>(LSE);
   long long c = 0;
+  // chunk sizes: the first two and the last two chunks of the call are a quarter and a half of
+  // G, so only a small chunk's inputs (at the start) and outputs (at the end) are exposed
+  const long long G4 = (G + 3) / 4, G2 = (G + 1) / 2;
   for (long long p0 = 0; cuda_ok && rc == TARA_OK && p0 < P; ++c) {
+    const long long left = P - p0;
     long long g = G;
-    if (p0 + g > P) g = P - p0;
+    if (P <= G) g = P;                     // one chunk: nothing to overlap
+    else if (left > G4 + G2 + G && p0 == 0) g = G4;
+    else if (left > G2 + G && p0 == G4 && G4 < G) g = G2;
+    else if (left <= G4) g = left;
+    else if (left <= G4 + G2) g = left - G4;
+    else if (left <= G4 + G2 + G) g = left - G4 - G2;
+    if (g > G) g = G;
+    if (g > left) g = left;
     if (strided && (p0 / H) != ((p0 + g - 1) / H)) g = (p0 / H + 1) * H - p0;   // stay in branch
     const int b = (int)(p0 / H);
     const int k = (int)(c & 1);
