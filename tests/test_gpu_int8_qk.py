@@ -154,3 +154,22 @@ def test_int8_stays_near_the_16bit_path():
     O16, L16 = run_gpu(w, q, k, v)
     assert (L8 - L16).abs().max().item() < 0.05
     assert (O8.float() - O16.float()).abs().mean().item() < 0.01
+
+
+def test_forward_per_branch_metadata():
+    # two branches with their own metadata (batch-strided) through the 8-bit path
+    import video_diffusion_attention_b200 as T
+    w = W.custom("q8pb", B=2, H=2, D=128, dtype="bf16", segments=_layout(tpf=40, frames=4),
+                 params=GAINS, seed_index=860)
+    q, k, v = (t.to(DEV) for t in W.make_qkv(w, DEV))
+    meta = T.pack_token_meta(w.segments)
+    N = len(meta["seg"])
+    stacked = {key: np.concatenate([val] * w.B) for key, val in meta.items()}
+    O, L = T.attn_forward(q, k, v, T.DeviceMeta(stacked, DEV, batch_stride=N, N=N),
+                          T.params_from(w.params, 1))
+    torch.cuda.synchronize()
+    assert T.device_status() == 0
+    rows = oracle.all_rows(w.B, w.H, w.N)
+    from parity_util import run_oracle_int8
+    Oref, Lref = run_oracle_int8(w, q, k, v, rows)
+    compare(w, O, L, rows, Oref, Lref, w.dtype)

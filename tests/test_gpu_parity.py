@@ -195,3 +195,25 @@ def test_calls_on_two_streams_do_not_share_summaries_concurrently():
     assert T.device_status() == 0
     for i, (O, L) in outs:
         assert torch.equal(O, ref[i][0]) and torch.equal(L, ref[i][1])
+
+
+@pytest.mark.parametrize("dtype,D", [("fp16", 128), ("bf16", 64)])
+def test_full_length_shot_other_dtype_and_head_dim(dtype, D):
+    # the 107,126-token layout at 8 heads in fp16, and with 64-wide heads, on sampled rows
+    base = W.get("micro")
+    w = W.custom("mic_%s_%d" % (dtype, D), B=1, H=4, D=D, dtype=dtype, segments=base.segments,
+                 params=W.Params(gain=(1.25, 0.75) + (1.0,) * 7), seed_index=950 + D)
+    _check(w, rows_from_sample(W.sample_rows(w, per_head=256)))
+
+
+def test_many_branch_head_planes():
+    # 3 x 700 (branch, head) planes: grid y/z well past one wave of CTAs per plane
+    segs = [W.Segment(W.TEXT, 1, 20), W.Segment(W.PICTURE, 1, 60, pic=1),
+            W.Segment(W.TARGET, 3, 50, frame_dt_s=4 / 24), W.Segment(W.GUIDE, 3, 50,
+                                                                      frame_dt_s=4 / 24)]
+    w = _small("bh", "bf16", 128, segs, GAINS, H=700, B=3, seed=960)
+    rng = np.random.Generator(np.random.PCG64(3))
+    b = rng.integers(0, 3, 600)
+    h = rng.integers(0, 700, 600)
+    i = rng.integers(0, w.N, 600)
+    _check(w, np.stack([b, h, i], axis=1).astype(np.int64))
