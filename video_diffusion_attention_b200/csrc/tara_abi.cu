@@ -234,6 +234,31 @@ int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& m
   return record_stop(stream);
 }
 
+// Kernel arguments shared by the workspace and the scratch-array entry points.
+TcArgs make_tc_args(const tara_token_meta* meta, tara_tensor* O, float* LSE, TileRec* recs,
+                    float4* keyinfo, int N, int H, int ntiles, int* status,
+                    const BiasParams& bp, const float* q_scale, const float* k_scale) {
+  TcArgs a;
+  a.O = O->ptr;
+  a.LSE = LSE;
+  a.seg = meta->seg;
+  a.time_s = meta->time_s;
+  a.m = meta->m;
+  a.recs = recs;
+  a.keyinfo = keyinfo;
+  a.meta_stride = (long long)meta->batch_stride;
+  a.N = N;
+  a.H = H;
+  a.ntiles = ntiles;
+  a.per_branch_meta = meta->batch_stride != 0 ? 1 : 0;
+  a.status = status;
+  a.bp = bp;
+  a.xm = ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride};
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  return a;
+}
+
 int validate(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
              const tara_token_meta* meta, const tara_params* p, const tara_tensor* O,
              const float* LSE) {
@@ -401,24 +426,7 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
       keyinfo);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
 
-  TcArgs a;
-  a.O = O->ptr;
-  a.LSE = LSE;
-  a.seg = meta->seg;
-  a.time_s = meta->time_s;
-  a.m = meta->m;
-  a.recs = recs;
-  a.keyinfo = keyinfo;
-  a.meta_stride = (long long)meta->batch_stride;
-  a.N = N;
-  a.H = H;
-  a.ntiles = ntiles;
-  a.per_branch_meta = meta->batch_stride != 0 ? 1 : 0;
-  a.status = st->status;
-  a.bp = bp;
-  a.xm = ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride};
-  a.q_scale = qs;
-  a.k_scale = ks;
+  const TcArgs a = make_tc_args(meta, O, LSE, recs, keyinfo, N, H, ntiles, st->status, bp, qs, ks);
   const bool bf16 = Q->dtype == TARA_BF16;
   if (q8)
     rc = bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
@@ -613,24 +621,8 @@ extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor
       keyinfo);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
 
-  TcArgs a;
-  a.O = O->ptr;
-  a.LSE = LSE;
-  a.seg = meta->seg;
-  a.time_s = meta->time_s;
-  a.m = meta->m;
-  a.recs = recs;
-  a.keyinfo = keyinfo;
-  a.meta_stride = (long long)meta->batch_stride;
-  a.N = N;
-  a.H = H;
-  a.ntiles = ntiles;
-  a.per_branch_meta = meta->batch_stride != 0 ? 1 : 0;
-  a.status = st->status;
-  a.bp = bp;
-  a.xm = ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride};
-  a.q_scale = nullptr;
-  a.k_scale = nullptr;
+  const TcArgs a =
+      make_tc_args(meta, O, LSE, recs, keyinfo, N, H, ntiles, st->status, bp, nullptr, nullptr);
   const bool bf16 = Q->dtype == TARA_BF16;
   if (D == 128)
     return bf16 ? launch_tc_static<true, 128>(mq, mk, mv, a, B, H, ntiles, stream)
