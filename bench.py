@@ -419,7 +419,8 @@ def main():
         q8_peak = 1.0 / (0.5 / (2.0 * p16) + 0.5 / p16)
         q8_ach = w.flops / (q8_line["kernel_ms"] * 1e-3) / 1e12
         q8_line["roofline"] = {"bound": "tensor", "achieved": q8_ach, "peak": q8_peak,
-                               "unit": "TFLOP/s", "frac": q8_ach / q8_peak, "traffic": None,
+                               "unit": "TFLOP/s", "frac": q8_ach / q8_peak,
+                               "traffic": recorded_traffic(w.name + "_int8"),
                                "peak_kind": "QK^T at 2 x measured sustained bf16 (nominal int8 "
                                             "ratio), PV at measured sustained bf16 (%s)" % peak_src}
     if mask_line is not None:
