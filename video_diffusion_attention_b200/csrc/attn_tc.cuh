@@ -57,6 +57,7 @@ struct TcShape {
   static constexpr int kSmemBytes = 1024 /*alignment slack*/ + 2 * kQKTileBytes +
                                     kStages * kTileBytes + kKeyBufBytes + kRowWBytes +
                                     kBarCount * 8 + 16;
+  static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
   static constexpr uint32_t kColS = 0;        // S_t at kColS + 128 t
   static constexpr uint32_t kColO = 256;      // O_t at kColO + D t
   static constexpr uint32_t kColP = 64;       // P_t at S_t + kColP
@@ -327,7 +328,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // dequantisation scales
     const float row_sl = kQ8 ? bp.scale_log2 * (row_ok ? args.q_scale[(long long)bh * N + row] : 0.0f)
                              : bp.scale_log2;
-    const float* kscale = args.k_scale + (long long)bh * args.ntiles;
+    const float* kscale = kQ8 ? args.k_scale + (long long)bh * args.ntiles : nullptr;
     float ks_next = kQ8 ? kscale[0] : 1.0f;
     // weights of the extra bindings for this row, one per Picture index (0 for index 0)
     float* wx = rowx + (t * kTile + r) * 17;
