@@ -14,14 +14,20 @@
 //
 // The bias never exists as an N x N tensor.  For each (query tile, key tile) pair the softmax
 // warps classify the pair from the two tile summaries: no bias, a constant -cap on every
-// target row, a constant m_row*ln(gain) on every target row, or per-edge evaluation from the
-// per-key records.  Constant biases fold into the per-row exponent offset, so they cost no
-// per-element work.  Logits are kept in log2 units: x = s*scale*log2(e) + bias*log2(e).
+// target row, a constant m_row*ln(gain) on every target row, one penalty per target row (a key
+// tile inside one guide frame), or per-edge evaluation from the per-key records.  Constant and
+// per-row biases fold into the per-row exponent offset, so they cost no per-element work.
+// Logits are kept in log2 units: x = s*scale*log2(e) + bias*log2(e).
 //
 // Online softmax: a thread holds its whole row of S (32x32b TMEM loads give one row per
-// thread), so the row max and sum need no cross-thread reduction.  The running max is only
-// raised when it grows by more than 2^8 in weight (P stays below 256), and only then is the
-// O row in TMEM rescaled, after the previous PV MMA has completed.
+// thread), so the row max and sum need no cross-thread reduction; exponents and sums run on
+// column pairs with packed f32x2 arithmetic.  The running max is only raised when it grows by
+// more than 2^8 in weight (P stays below 256), and only then is the O row in TMEM rescaled,
+// after the previous PV MMA has completed.
+//
+// kQ8 (the INT8 QK^T variant): Q and K arrive as 8-bit codes with per-row and per-key-tile
+// scales, QK^T runs as tcgen05.mma.kind::i8 into s32 S, and the scales join the softmax scale
+// in the per-tile row multiplier.
 #pragma once
 
 #include "sm100_ptx.cuh"
