@@ -66,13 +66,14 @@ KERNEL_SOURCES = ("attn_tc.cuh", "sm100_ptx.cuh", "tara_common.cuh")
 
 
 def kernel_source_hash() -> str:
-    """sha256 (first 16 hex digits) of the kernel's device sources with // comments and
-    trailing blanks removed: edits to comments leave it unchanged, edits to code do not."""
+    """sha256 (first 16 hex digits) of the kernel's device sources with // comments, trailing
+    blanks and empty lines removed: edits to comments leave it unchanged, edits to code do not."""
     import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         with open(os.path.join(CSRC, f)) as fh:
-            code = "\n".join(re.sub(r"//.*$", "", line).rstrip() for line in fh.read().splitlines())
+            lines = (re.sub(r"//.*$", "", line).rstrip() for line in fh.read().splitlines())
+            code = "\n".join(line for line in lines if line)
         h.update(f.encode() + code.encode())
     return h.hexdigest()[:16]
 
