@@ -83,7 +83,8 @@ typedef enum {
 
 typedef enum { TARA_BF16 = 0, TARA_FP16 = 1, TARA_FP32 = 2 } tara_dtype;
 
-/* A dense tensor [B][H][N][D], row-major and contiguous, in device memory. */
+/* A dense tensor [B][H][N][D], row-major and contiguous, in device memory (host memory for
+ * tara_attn_forward_host). */
 typedef struct {
   void*      ptr;
   tara_dtype dtype;
@@ -91,7 +92,7 @@ typedef struct {
 } tara_tensor;
 
 /* Per-token metadata of the packed sequence, four device arrays of length N each
- * (structure of arrays).  batch_stride = 0: one set shared by all B branches (the CFG
+ * (structure of arrays; host arrays for tara_attn_forward_host).  batch_stride = 0: one set shared by all B branches (the CFG
  * branches of one shot share their packing); otherwise set b starts at element
  * b * batch_stride of every array and there are B sets.
  *   seg    : tara_seg value per token
