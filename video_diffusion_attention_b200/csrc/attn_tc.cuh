@@ -400,10 +400,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!(ok = warp_wait(&s_full[t], (uint32_t)j & 1u, abort_flag, kWaitLimitNs))) break;
       tc_fence_after();
       uint32_t s[128];
-      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_ld128(tS, s);
       tmem_ld_wait();
       reg_fence<128>(s);
       const int nv = (int)kr.nvalid;
