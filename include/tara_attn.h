@@ -174,16 +174,19 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
  * extra_m) in HOST memory; pinned memory (cudaHostAlloc / cudaHostRegister) lets the copies
  * overlap the kernels, pageable memory works but serialises them.  The pages have no
  * counterpart: it is the runtime around the kernel for callers whose tensors live on the host.
- *   The B*H (branch, head) planes are processed in chunks of consecutive planes (about 1 GiB of
- *   Q, K, V and O each, within one branch when the metadata is per branch): per chunk, the
- *   host->device copies of Q, K, V run on one internal stream, the attention
- *   (tara_attn_forward on device chunk buffers) on a second, and the device->host copies of O
- *   and LSE on a third, with two chunk buffer sets alternating, so transfers overlap kernels.
+ *   The B*H (branch, head) planes are processed in chunks of consecutive planes (at most about
+ *   1 GiB of Q, K, V and O each, within one branch when the metadata is per branch; 1, 2, 4,
+ *   ... planes at the start and the same ramp reversed at the end): per chunk, the
+ *   host->device copies of Q, K, V run on one internal stream, the attention (the kernels of
+ *   tara_attn_forward on device chunk buffers) on one of two internal compute streams, and the
+ *   device->host copies of O and LSE on a fourth.  Two chunk buffer sets, each with its own
+ *   workspace, and the two compute streams alternate between consecutive chunks, so transfers
+ *   overlap kernels and one chunk's kernel fills the SMs the previous one's last wave leaves.
  *   Ordering: everything runs after the work already queued on `stream`, and `stream` waits
  *   for the last copy; the call itself does not block the host.  The host buffers must stay
  *   valid and unmodified until `stream` has completed (as with cudaMemcpyAsync).
- *   Device memory: the metadata plus two chunk sets, cached per device and grown with
- *   cudaMalloc (a growth synchronises the device).  A kernel-event pair pending for the
+ *   Device memory: the metadata plus two chunk sets with their workspaces, cached per device
+ *   and grown with cudaMalloc (a growth synchronises the device).  A kernel-event pair pending for the
  *   calling thread (tara_set_kernel_events) is dropped.
  * Same arguments and checks as tara_attn_forward (shapes, dtypes, parameters, extra
  * bindings) except that pointers are host pointers with no alignment requirement.

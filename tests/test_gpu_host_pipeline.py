@@ -2,8 +2,9 @@
 
 Every (branch, head) plane is computed by the same kernels as tara_attn_forward on device
 buffers, so the chunked three-stream pipeline must reproduce the device-buffer result bit for
-bit, across chunk boundaries, branch cuts of per-branch metadata, extra bindings and the INT8
-QK^T variant.
+bit, across chunk boundaries (a 1, 2, 4, ... ramp at both ends, kernels of consecutive chunks
+on alternating streams), branch cuts of per-branch metadata, extra bindings and the INT8 QK^T
+variant.
 """
 import numpy as np
 import pytest
@@ -46,9 +47,20 @@ def test_single_chunk_bf16_int8():
     _both(W.get("medium"), qk_int8=1)
 
 
-def test_full_shot_seven_chunks():
-    # 56 heads of 27.4 MB planes: chunks of 9 planes, the last one short
+def test_full_shot_ramped_chunks():
+    # 56 heads of 27.4 MB planes: chunks of 1, 2, 4, 8, 9, 9, 8, 8, 4, 2, 1 planes
     _both(W.get("full"))
+
+
+def test_ramp_cut_at_branches_int8():
+    # 2 branches x 5 heads with per-branch metadata: the ramp 1, 2, 4, 2, 1 is cut at the
+    # branch boundary (planes 3-6 become 3-4 and 5-6); INT8 quantisation per chunk
+    w = W.custom("hramp", B=2, H=5, D=128, dtype="bf16", segments=[
+        W.Segment(W.TEXT, 1, 70), W.Segment(W.PICTURE, 1, 200, pic=1),
+        W.Segment(W.TARGET, 4, 120, frame_dt_s=4 / 24, mask=W.uniform_mask(5, 120)),
+        W.Segment(W.GUIDE, 4, 97, frame_dt_s=4 / 24), W.Segment(W.AUDIO, 1, 33)],
+        params=W.Params(gain=(1.4,) + (1.0,) * 8), seed_index=910)
+    _both(w, per_branch_meta=True, qk_int8=1)
 
 
 def test_per_branch_metadata_chunks_cut_at_branches():

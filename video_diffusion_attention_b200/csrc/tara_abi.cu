@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "tara_attn.h"
+#include "forward_internal.h"
 #include "param_checks.h"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
@@ -305,7 +306,137 @@ int validate(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
   return TARA_OK;
 }
 
+// Workspace of one tensor-core forward call: tile records and per-key records of every
+// metadata set, then (qk_int8 only) the 8-bit copies of Q and K and their scales.
+struct WsLayout {
+  int nsets;
+  size_t rec, key, code, qs, ks, total;
+};
+
+WsLayout ws_layout(const tara_tensor* Q, const tara_token_meta* meta, const tara_params* p) {
+  WsLayout L;
+  const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
+  const int ntiles = (N + kTile - 1) / kTile;
+  L.nsets = meta->batch_stride != 0 ? B : 1;
+  L.rec = round_up((size_t)L.nsets * ntiles * sizeof(TileRec), 256);
+  L.key = round_up((size_t)L.nsets * N * sizeof(float4), 256);
+  const bool q8 = p->qk_int8 != 0;
+  L.code = q8 ? round_up((size_t)B * H * N * D, 256) : 0;
+  L.qs = q8 ? round_up((size_t)B * H * N * sizeof(float), 256) : 0;
+  L.ks = q8 ? round_up((size_t)B * H * ntiles * sizeof(float), 256) : 0;
+  L.total = Q->dtype == TARA_FP32 ? 0 : L.rec + L.key + 2 * L.code + L.qs + L.ks;
+  return L;
+}
+
+// The forward pass after argument checks, with g_mu held.  ws_ext == nullptr: the device's
+// shared workspace, ordered against every other call through ws_free.  Otherwise the caller's
+// workspace of ws_ext_bytes (at least ws_layout(...).total of the shape), which the caller orders.
+int forward_locked(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
+                   const tara_token_meta* meta, const tara_params* p, tara_tensor* O, float* LSE,
+                   cudaStream_t stream, void* ws_ext, size_t ws_ext_bytes) {
+  int rc = TARA_OK;
+  const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
+  const BiasParams bp = make_bias_params(p, D);
+
+  if (Q->dtype == TARA_FP32) {
+    DeviceState* st = nullptr;
+    if ((rc = device_state(0, &st)) != TARA_OK) return rc;
+    const size_t smem = (size_t)(2 * kSimtChunk * (D + 1) + kSimtRows * D) * sizeof(float);
+    if (!st->simt_attr_set) {
+      if (cudaFuncSetAttribute(attn_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)((2 * kSimtChunk * (kSimtMaxD + 1) + kSimtRows * kSimtMaxD) *
+                                     sizeof(float))) != cudaSuccess)
+        return TARA_ERR_CUDA;
+      st->simt_attr_set = true;
+    }
+    dim3 grid((unsigned)((N + kSimtRows - 1) / kSimtRows), (unsigned)H, (unsigned)B);
+    if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
+    attn_simt_kernel<<<grid, kSimtRows * 32, smem, stream>>>(
+        static_cast<const float*>(Q->ptr), static_cast<const float*>(K->ptr),
+        static_cast<const float*>(V->ptr), static_cast<float*>(O->ptr), LSE, meta->seg,
+        meta->time_s, meta->pic, meta->m, (long long)meta->batch_stride, H, N, D, bp,
+        ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride});
+    if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
+    return record_stop(stream);
+  }
+
+  if ((rc = get_encode_fn()) != TARA_OK) return rc;
+  const int ntiles = (N + kTile - 1) / kTile;
+  const WsLayout L = ws_layout(Q, meta, p);
+  const bool q8 = p->qk_int8 != 0;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(ws_ext ? 0 : L.total, &st)) != TARA_OK) return rc;
+  if (ws_ext && ws_ext_bytes < L.total) return TARA_ERR_TOO_LARGE;
+  char* ws = static_cast<char*>(ws_ext ? ws_ext : st->ws);
+  TileRec* recs = reinterpret_cast<TileRec*>(ws);
+  float4* keyinfo = reinterpret_cast<float4*>(ws + L.rec);
+  int8_t* qc = reinterpret_cast<int8_t*>(ws + L.rec + L.key);
+  int8_t* kc = qc + L.code;
+  float* qs = reinterpret_cast<float*>(ws + L.rec + L.key + 2 * L.code);
+  float* ks = reinterpret_cast<float*>(ws + L.rec + L.key + 2 * L.code + L.qs);
+
+  // wait for the previous call's kernels to finish reading the shared workspace (not while the
+  // stream is being captured: a captured wait on an event recorded outside the graph is not
+  // allowed; a caller-owned workspace is ordered by its owner)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return TARA_ERR_CUDA;
+  const bool order_ws = cap == cudaStreamCaptureStatusNone && ws_ext == nullptr;
+  if (order_ws) {
+    if (!st->ws_free && cudaEventCreateWithFlags(&st->ws_free, cudaEventDisableTiming) != cudaSuccess)
+      return TARA_ERR_CUDA;
+    if (cudaStreamWaitEvent(stream, st->ws_free, 0) != cudaSuccess) return TARA_ERR_CUDA;
+  }
+
+  CUtensorMap mq, mk, mv;
+  if (q8) {
+    if (encode_q8_map(&mq, qc, B * H, N, D) != TARA_OK ||
+        encode_q8_map(&mk, kc, B * H, N, D) != TARA_OK || encode_qkv_map(&mv, V) != TARA_OK)
+      return TARA_ERR_CUDA;
+    if ((rc = launch_quant(Q, K, qc, qs, kc, ks, stream)) != TARA_OK) return rc;
+  } else if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K) != TARA_OK ||
+             encode_qkv_map(&mv, V) != TARA_OK) {
+    return TARA_ERR_CUDA;
+  }
+
+  tile_summary_kernel<<<dim3((unsigned)ntiles, (unsigned)L.nsets), 128, 0, stream>>>(
+      meta->seg, meta->time_s, meta->pic, N, (long long)meta->batch_stride, ntiles, bp, recs,
+      keyinfo);
+  if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
+
+  const TcArgs a = make_tc_args(meta, O, LSE, recs, keyinfo, N, H, ntiles, st->status, bp, qs, ks);
+  const bool bf16 = Q->dtype == TARA_BF16;
+  if (q8)
+    rc = bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
+              : launch_tc<false, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st);
+  else if (D == 128)
+    rc = bf16 ? launch_tc<true, 128>(mq, mk, mv, a, B, H, ntiles, stream, st)
+              : launch_tc<false, 128>(mq, mk, mv, a, B, H, ntiles, stream, st);
+  else
+    rc = bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
+              : launch_tc<false, 64>(mq, mk, mv, a, B, H, ntiles, stream, st);
+  if (rc == TARA_OK && order_ws && cudaEventRecord(st->ws_free, stream) != cudaSuccess)
+    return TARA_ERR_CUDA;
+  return rc;
+}
+
 }  // namespace
+
+size_t forward_workspace_bytes(const tara_tensor* Q, const tara_token_meta* meta,
+                               const tara_params* p) {
+  return ws_layout(Q, meta, p).total;
+}
+
+int forward_with_workspace(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
+                           const tara_token_meta* meta, const tara_params* p, tara_tensor* O,
+                           float* LSE, void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate(Q, K, V, meta, p, O, LSE);
+  if (rc != TARA_OK) return rc;
+  if (Q->dtype != TARA_FP32 && !ws) return TARA_ERR_NULL;
+  if (!aligned16(ws)) return TARA_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  return forward_locked(Q, K, V, meta, p, O, LSE, static_cast<cudaStream_t>(stream), ws, ws_bytes);
+}
+
 }  // namespace tara
 
 using namespace tara;
@@ -350,96 +481,8 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
                       float* LSE, void* stream_) {
   int rc = validate(Q, K, V, meta, p, O, LSE);
   if (rc != TARA_OK) return rc;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
-  const BiasParams bp = make_bias_params(p, D);
-
   std::lock_guard<std::mutex> lock(g_mu);
-  if (Q->dtype == TARA_FP32) {
-    DeviceState* st = nullptr;
-    if ((rc = device_state(0, &st)) != TARA_OK) return rc;
-    const size_t smem = (size_t)(2 * kSimtChunk * (D + 1) + kSimtRows * D) * sizeof(float);
-    if (!st->simt_attr_set) {
-      if (cudaFuncSetAttribute(attn_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)((2 * kSimtChunk * (kSimtMaxD + 1) + kSimtRows * kSimtMaxD) *
-                                     sizeof(float))) != cudaSuccess)
-        return TARA_ERR_CUDA;
-      st->simt_attr_set = true;
-    }
-    dim3 grid((unsigned)((N + kSimtRows - 1) / kSimtRows), (unsigned)H, (unsigned)B);
-    if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
-    attn_simt_kernel<<<grid, kSimtRows * 32, smem, stream>>>(
-        static_cast<const float*>(Q->ptr), static_cast<const float*>(K->ptr),
-        static_cast<const float*>(V->ptr), static_cast<float*>(O->ptr), LSE, meta->seg,
-        meta->time_s, meta->pic, meta->m, (long long)meta->batch_stride, H, N, D, bp,
-        ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride});
-    if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
-    return record_stop(stream);
-  }
-
-  if ((rc = get_encode_fn()) != TARA_OK) return rc;
-  const int ntiles = (N + kTile - 1) / kTile;
-  const int nsets = meta->batch_stride != 0 ? B : 1;
-  const size_t rec_bytes = round_up((size_t)nsets * ntiles * sizeof(TileRec), 256);
-  const size_t key_bytes = round_up((size_t)nsets * N * sizeof(float4), 256);
-  // 8-bit copies of Q and K with their scales (qk_int8 only)
-  const bool q8 = p->qk_int8 != 0;
-  const size_t code_bytes = q8 ? round_up((size_t)B * H * N * D, 256) : 0;
-  const size_t qs_bytes = q8 ? round_up((size_t)B * H * N * sizeof(float), 256) : 0;
-  const size_t ks_bytes = q8 ? round_up((size_t)B * H * ntiles * sizeof(float), 256) : 0;
-  DeviceState* st = nullptr;
-  if ((rc = device_state(rec_bytes + key_bytes + 2 * code_bytes + qs_bytes + ks_bytes, &st)) !=
-      TARA_OK)
-    return rc;
-  char* ws = static_cast<char*>(st->ws);
-  TileRec* recs = reinterpret_cast<TileRec*>(ws);
-  float4* keyinfo = reinterpret_cast<float4*>(ws + rec_bytes);
-  int8_t* qc = reinterpret_cast<int8_t*>(ws + rec_bytes + key_bytes);
-  int8_t* kc = qc + code_bytes;
-  float* qs = reinterpret_cast<float*>(ws + rec_bytes + key_bytes + 2 * code_bytes);
-  float* ks = reinterpret_cast<float*>(ws + rec_bytes + key_bytes + 2 * code_bytes + qs_bytes);
-
-  // wait for the previous call's kernels to finish reading the workspace (not while the stream
-  // is being captured: a captured wait on an event recorded outside the graph is not allowed)
-  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return TARA_ERR_CUDA;
-  const bool order_ws = cap == cudaStreamCaptureStatusNone;
-  if (order_ws) {
-    if (!st->ws_free && cudaEventCreateWithFlags(&st->ws_free, cudaEventDisableTiming) != cudaSuccess)
-      return TARA_ERR_CUDA;
-    if (cudaStreamWaitEvent(stream, st->ws_free, 0) != cudaSuccess) return TARA_ERR_CUDA;
-  }
-
-  CUtensorMap mq, mk, mv;
-  if (q8) {
-    if (encode_q8_map(&mq, qc, B * H, N, D) != TARA_OK ||
-        encode_q8_map(&mk, kc, B * H, N, D) != TARA_OK || encode_qkv_map(&mv, V) != TARA_OK)
-      return TARA_ERR_CUDA;
-    if ((rc = launch_quant(Q, K, qc, qs, kc, ks, stream)) != TARA_OK) return rc;
-  } else if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K) != TARA_OK ||
-             encode_qkv_map(&mv, V) != TARA_OK) {
-    return TARA_ERR_CUDA;
-  }
-
-  tile_summary_kernel<<<dim3((unsigned)ntiles, (unsigned)nsets), 128, 0, stream>>>(
-      meta->seg, meta->time_s, meta->pic, N, (long long)meta->batch_stride, ntiles, bp, recs,
-      keyinfo);
-  if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
-
-  const TcArgs a = make_tc_args(meta, O, LSE, recs, keyinfo, N, H, ntiles, st->status, bp, qs, ks);
-  const bool bf16 = Q->dtype == TARA_BF16;
-  if (q8)
-    rc = bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
-              : launch_tc<false, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st);
-  else if (D == 128)
-    rc = bf16 ? launch_tc<true, 128>(mq, mk, mv, a, B, H, ntiles, stream, st)
-              : launch_tc<false, 128>(mq, mk, mv, a, B, H, ntiles, stream, st);
-  else
-    rc = bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
-              : launch_tc<false, 64>(mq, mk, mv, a, B, H, ntiles, stream, st);
-  if (rc == TARA_OK && order_ws && cudaEventRecord(st->ws_free, stream) != cudaSuccess)
-    return TARA_ERR_CUDA;
-  return rc;
+  return forward_locked(Q, K, V, meta, p, O, LSE, static_cast<cudaStream_t>(stream_), nullptr, 0);
 }
 
 int tara_quantize_qk_int8(const tara_tensor* Q, const tara_tensor* K, int8_t* q_codes,
