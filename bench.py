@@ -375,15 +375,18 @@ def main():
         mo = torch.empty((tgt[0].frames, 40, 50), dtype=torch.float32, device=dev)
         for _ in range(3):
             T.prepare_target_mask(px, 107, 4, tgt[0].frames, 40, 50, out=mo, stream=stream)
-        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # one event pair around each launch: a ~45 us kernel is shorter than the Python call
+        # that launches it, so events around a back-to-back loop would time the host instead
         reps = 20
+        mev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
         torch.cuda.synchronize(dev)
-        m0.record(stream)
-        for _ in range(reps):
+        for a, b in mev:
+            a.record(stream)
             T.prepare_target_mask(px, 107, 4, tgt[0].frames, 40, 50, out=mo, stream=stream)
-        m1.record(stream)
+            b.record(stream)
         torch.cuda.synchronize(dev)
-        mms = m0.elapsed_time(m1) / reps
+        mms = statistics.median(a.elapsed_time(b) for a, b in mev)
         mbytes = px.numel() * 4 + mo.numel() * 4
         mask_line = {"kernel": "target_mask_narrow_kernel (rows <= 1024 px)", "workload": "107x544x928 fp32 pixel mask -> "
                      "%dx40x50 target weights" % tgt[0].frames, "ms": mms, "bound": "hbm",

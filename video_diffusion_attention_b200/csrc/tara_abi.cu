@@ -524,10 +524,10 @@ int tara_prepare_target_mask(const float* mask, int32_t F_in, int32_t Hp, int32_
   if ((reinterpret_cast<uintptr_t>(mask) & 3u) != 0 || (reinterpret_cast<uintptr_t>(m_out) & 3u) != 0)
     return TARA_ERR_ALIGN;
   dim3 grid((unsigned)Hq, (unsigned)(F_in > 1 ? F_lat : 1));
-  const bool narrow = Wp <= 4 * kMaskThreads && Wp % 4 == 0 &&
+  const bool narrow = Wp <= 8 * kMaskNarrowThreads && Wp % 4 == 0 &&
                       (reinterpret_cast<uintptr_t>(mask) & 15u) == 0;
   if (narrow)
-    target_mask_narrow_kernel<<<grid, kMaskThreads, (size_t)Wq * sizeof(float),
+    target_mask_narrow_kernel<<<grid, kMaskNarrowThreads, (size_t)Wq * sizeof(float),
                                 static_cast<cudaStream_t>(stream_)>>>(
         mask, F_in, Hp, Wp, shot_len, frames_per_latent, F_lat, Hq, Wq, m_out);
   else

@@ -105,17 +105,36 @@ target_mask_kernel(const float* __restrict__ mask, int F_in, int Hp, int Wp, int
   }
 }
 
-// Narrow rows (Wp <= 1024, every pixel row 16-byte aligned): thread t owns columns 4t..4t+3,
-// one 16-byte load per pixel row, and walks the (pixel frame, pixel row) pairs of its cell
-// row eight at a time so that eight loads are in flight per thread.
-__global__ void __launch_bounds__(kMaskThreads)
+// Adds the weighted column sums of pixel columns c..c+3 into the cells they overlap.
+__device__ __forceinline__ void add_column_group(float* cell_acc, float4 cs, int c, int Wp,
+                                                 int Wq) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float vk = k == 0 ? cs.x : k == 1 ? cs.y : k == 2 ? cs.z : cs.w;
+    const long long clo = (long long)(c + k) * Wq, chi = clo + Wq;
+    for (int x = (int)(clo / Wp); x < Wq && (long long)x * Wp < chi; ++x) {
+      const long long xlo = (long long)x * Wp;
+      const float wx = (float)(min(xlo + Wp, chi) - max(xlo, clo));
+      atomicAdd(&cell_acc[x], wx * vk);
+    }
+  }
+}
+
+// Narrow rows (Wp <= 1024, every pixel row 16-byte aligned): 128 threads, thread t owns the
+// 16-byte column groups t and t + 128 (one load each per pixel row), so a CTA needs few
+// registers and the whole grid of a shot is resident at once.  The (pixel frame, pixel row)
+// pairs of the cell row are walked with an incremented index pair (no division in the loop),
+// four at a time, so eight loads are in flight per thread.
+constexpr int kMaskNarrowThreads = 128;
+
+__global__ void __launch_bounds__(kMaskNarrowThreads)
 target_mask_narrow_kernel(const float* __restrict__ mask, int F_in, int Hp, int Wp, int L,
                           int tau, int F_lat, int Hq, int Wq, float* __restrict__ out) {
   extern __shared__ float cell_acc[];   // [Wq]
   const int y = blockIdx.x;
   const int f = blockIdx.y;
   const int tid = threadIdx.x;
-  for (int x = tid; x < Wq; x += kMaskThreads) cell_acc[x] = 0.0f;
+  for (int x = tid; x < Wq; x += kMaskNarrowThreads) cell_acc[x] = 0.0f;
   __syncthreads();
 
   const long long ylo = (long long)y * Hp, yhi = (long long)(y + 1) * Hp;
@@ -126,38 +145,41 @@ target_mask_narrow_kernel(const float* __restrict__ mask, int F_in, int Hp, int 
     t0 = f * tau;
     t1 = min(t0 + tau, L);
   }
-  const int nr = r1 - r0;
-  const int npairs = (t1 - t0) * nr;
-  const int c = tid * 4;
-  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  if (c < Wp) {
-#pragma unroll 8
+  const int npairs = (t1 - t0) * (r1 - r0);
+  const int c0 = tid * 4, c1 = (tid + kMaskNarrowThreads) * 4;
+  const bool has1 = c1 < Wp;
+  float4 a0 = make_float4(0.0f, 0.0f, 0.0f, 0.0f), a1 = a0;
+  if (c0 < Wp) {
+    int t = t0, r = r0;
+#pragma unroll 4
     for (int i = 0; i < npairs; ++i) {
-      const int t = t0 + i / nr;
-      const int r = r0 + i % nr;
       const long long rlo = (long long)r * Hq;
       const float wy = (float)(min(yhi, rlo + Hq) - max(ylo, rlo));
-      const float4 v = __ldg(reinterpret_cast<const float4*>(mask + ((long long)t * Hp + r) * Wp + c));
-      acc.x = fmaf(wy, v.x, acc.x);
-      acc.y = fmaf(wy, v.y, acc.y);
-      acc.z = fmaf(wy, v.z, acc.z);
-      acc.w = fmaf(wy, v.w, acc.w);
-    }
-    const float cs[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const long long clo = (long long)(c + k) * Wq, chi = clo + Wq;
-      for (int x = (int)(clo / Wp); x < Wq && (long long)x * Wp < chi; ++x) {
-        const long long xlo = (long long)x * Wp;
-        const float wx = (float)(min(xlo + Wp, chi) - max(xlo, clo));
-        atomicAdd(&cell_acc[x], wx * cs[k]);
+      const float* row = mask + ((long long)t * Hp + r) * Wp;
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row + c0));
+      a0.x = fmaf(wy, v.x, a0.x);
+      a0.y = fmaf(wy, v.y, a0.y);
+      a0.z = fmaf(wy, v.z, a0.z);
+      a0.w = fmaf(wy, v.w, a0.w);
+      if (has1) {
+        const float4 u = __ldg(reinterpret_cast<const float4*>(row + c1));
+        a1.x = fmaf(wy, u.x, a1.x);
+        a1.y = fmaf(wy, u.y, a1.y);
+        a1.z = fmaf(wy, u.z, a1.z);
+        a1.w = fmaf(wy, u.w, a1.w);
+      }
+      if (++r == r1) {
+        r = r0;
+        ++t;
       }
     }
+    add_column_group(cell_acc, a0, c0, Wp, Wq);
+    if (has1) add_column_group(cell_acc, a1, c1, Wp, Wq);
   }
   __syncthreads();
 
   const float norm = 1.0f / ((float)Hp * (float)Wp * (float)(t1 - t0));
-  for (int x = tid; x < Wq; x += kMaskThreads) {
+  for (int x = tid; x < Wq; x += kMaskNarrowThreads) {
     const float v = cell_acc[x] * norm;
     if (F_in > 1) {
       out[((long long)f * Hq + y) * Wq + x] = v;
