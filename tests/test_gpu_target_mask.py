@@ -20,6 +20,8 @@ CASES = [
     (107, 720, 1280, 107, 4, 27, 40, 50),    # pixel-resolution mask of the full shot
     (107, 544, 928, 107, 4, 27, 40, 50),     # the pages' user-run resolution (narrow rows)
     (22, 33, 1024, 22, 4, 6, 7, 50),         # widest narrow-row case
+    (22, 33, 516, 22, 4, 6, 7, 50),          # narrow rows: only thread 0 has a second column group
+    (1, 17, 508, 107, 4, 26, 5, 9),          # static narrow mask, no second column group
     (22, 33, 1028, 22, 4, 6, 7, 50),         # just past it: the general kernel
 ]
 
