@@ -71,7 +71,8 @@ def test_temporal_spans_and_static_mask():
         expect = vals[f * tau:min(f * tau + tau, L)].mean()
         assert np.allclose(out[f], expect, atol=1e-15)
     assert F_lat * tau > L               # the last span is short (3 frames): still averaged
-    static = oracle.prepare_target_mask(m[:1], L, 26, 4, 2, 2)
-    assert np.allclose(static, vals[0])
+    # a one-frame mask applies unchanged to every latent frame (frame 5: not all zeros)
+    static = oracle.prepare_target_mask(m[5:6], L, 26, 4, 2, 2)
+    assert static.shape == (26, 2, 2) and np.allclose(static, vals[5]) and vals[5] > 0
     with pytest.raises(ValueError):
         oracle.prepare_target_mask(m, L, 28, 4, 2, 2)   # latent frame 27 starts past the shot
