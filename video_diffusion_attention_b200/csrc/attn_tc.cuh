@@ -278,8 +278,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int kk = 0; kk < kTile / 16; ++kk)
               umma_ts(d_o, a_p + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                       (j > 1 || kk > 0) ? 1u : 0u);
-            umma_commit(&pv_done[t]);
-            if (t == 1) umma_commit(&kv_empty[vslot]);
           }
           if (j < nk) {
             const uint32_t d_s = tmem + S::kColS + t * 128;
@@ -299,8 +297,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               }
             }
             umma_commit(&s_full[t]);
-            if (t == 1) umma_commit(&kv_empty[kslot]);
           }
+          // PV's completion and the V slot's release are committed after the next QK^T is
+          // issued: a commit costs the issuing thread ~55 cycles, and here it is off the
+          // P -> PV -> QK^T -> S path (the only waiters on pv_done waited for that QK^T
+          // already, through s_full, or are the epilogue, where no QK^T follows)
+          if (j > 0) {
+            umma_commit(&pv_done[t]);
+            if (t == 1) umma_commit(&kv_empty[(2 * (j - 1) + 1) % NS]);
+          }
+          if (j < nk && t == 1) umma_commit(&kv_empty[kslot]);
         }
       }
       // every MMA issued above completes before tensor memory is released
