@@ -40,6 +40,11 @@ MUTANTS = {
     "signed time difference": ("double dt = fabs((double)time_s[i] - (double)time_s[j]);",
                                "double dt = (double)time_s[i] - (double)time_s[j];"),
     "guide/picture roles swapped": ("if (seg[j] == ROLE_GUIDE) {", "if (seg[j] == ROLE_PICTURE) {"),
+    # each rule parameter replaced by its printed default
+    "falloff hard-coded to its default": ("x = x / falloff;", "x = x / 0.25;"),
+    "window hard-coded to its default": ("double x = dt - window;", "double x = dt - 0.20;"),
+    "strength hard-coded to its default": ("double p = strength * x * x;", "double p = 2.0 * x * x;"),
+    "cap hard-coded to its default": ("return p < cap ? p : cap;", "return p < 6.0 ? p : 6.0;"),
 }
 
 

@@ -114,6 +114,84 @@ def test_penalty_grows_quadratically_then_caps(golden_rule):
         2 * oracle.penalty(w + 0.05, w, f, s, c), rel=1e-12)
 
 
+def test_penalty_on_default_latent_grid(golden_rule):
+    # P1: the rule at its printed defaults on the 4/24 s latent clock, against the exact
+    # rational values derived by hand in the golden file ("The temporal rule")
+    w, f, s, c = (golden_rule[k][0] for k in ("window", "falloff", "strength", "cap"))
+    for d in range(5):
+        val, tol = golden_rule["penalty_default_d%d" % d]
+        assert abs(oracle.penalty(d / 6.0, w, f, s, c) - val) <= tol, d
+
+
+def _ragged_rule(golden_rule):
+    return tuple(golden_rule["ragged_" + k][0] for k in ("window", "falloff", "strength", "cap"))
+
+
+def test_penalty_at_non_default_parameters(golden_rule):
+    # P2: every parameter away from its default (the ragged workload's window 0.10, falloff
+    # 0.40, strength 3.0, cap 8.0), with the guide clock offset by 1/24 s; exact values
+    # derived by hand in the golden file.  A rule that ignores any one of the four
+    # parameters in favour of its default misses several of them.
+    w, f, s, c = _ragged_rule(golden_rule)
+    for d in range(-4, 6):
+        key = "penalty_ragged_d%s" % (("m%d" % -d) if d < 0 else str(d))
+        val, tol = golden_rule[key]
+        dt = abs(4 * d - 1) / 24.0
+        assert abs(oracle.penalty(dt, w, f, s, c) - val) <= tol, d
+
+
+def test_cap_point_at_non_default_parameters(golden_rule):
+    # The first delay at which the penalty equals the cap: window + falloff*sqrt(cap/strength)
+    # (inverting the quadratic branch of "The temporal rule").  Checked against the golden
+    # value for the ragged parameters and, by bisection, for parameter sets where each of
+    # the four moves on its own.
+    w, f, s, c = _ragged_rule(golden_rule)
+    sets = [(w, f, s, c, golden_rule["ragged_cap_reached_at_s"][0]),
+            (0.05, 0.25, 2.0, 6.0, None), (0.20, 0.60, 2.0, 6.0, None),
+            (0.20, 0.25, 5.0, 6.0, None), (0.20, 0.25, 2.0, 1.5, None)]
+    for (ww, ff, ss, cc, printed) in sets:
+        t_star = ww + ff * math.sqrt(cc / ss)
+        if printed is not None:
+            assert abs(t_star - printed) <= 1e-11
+        lo, hi = ww, 100.0
+        for _ in range(200):
+            mid = 0.5 * (lo + hi)
+            if oracle.penalty(mid, ww, ff, ss, cc) >= cc:
+                hi = mid
+            else:
+                lo = mid
+        assert abs(hi - t_star) <= 1e-12, (ww, ff, ss, cc)
+
+
+def test_logit_row_at_non_default_parameters(golden_rule):
+    # The oracle's dense logit row of one target query with Q = 0 (so every dot product is
+    # 0): its guide entries are minus the ragged penalties above, its picture entries
+    # m*ln(gain) ("BFS H3 Reference Attention Binding (Experimental)", "The exact rule") and
+    # every other entry 0.  Times pass through the packer's float32 clock, which moves dt by
+    # under 1e-7 s; the penalty's slope (< 30 per second here) bounds the effect.
+    w, f, s, c = _ragged_rule(golden_rule)
+    off = golden_rule["ragged_guide_offset_s"][0]
+    segs = [W.Segment(W.TEXT, 1, 2), W.Segment(W.PICTURE, 1, 3, pic=1),
+            W.Segment(W.TARGET, 10, 1, frame_dt_s=4 / 24,
+                      mask=np.full(10, 0.625, dtype=np.float32)),
+            W.Segment(W.GUIDE, 10, 1, t0_s=off, frame_dt_s=4 / 24), W.Segment(W.AUDIO, 1, 2)]
+    meta = oracle.pack_token_meta(segs)
+    N = len(meta["seg"])
+    q = np.zeros((1, 1, N, 8))
+    k = np.random.Generator(np.random.PCG64(5)).standard_normal((1, 1, N, 8))
+    p = W.Params(window=w, falloff=f, strength=s, cap=c, gain=(1.5,) + (1.0,) * 8)
+    t0 = 5                                  # the query: target frame 5
+    row = oracle.logit_row(q, k, "fp64", meta, p, 0, 0, t0 + 5, params_as_float32=False)
+    tgt = np.arange(5, 15)
+    gde = np.arange(15, 25)
+    for g, j in enumerate(gde):
+        d = 5 - g
+        key = "penalty_ragged_d%s" % (("m%d" % -d) if d < 0 else str(d))
+        assert abs(row[j] + golden_rule[key][0]) <= 1e-6, d
+    assert np.allclose(row[2:5], 0.625 * math.log(1.5), rtol=0, atol=1e-7)
+    assert np.all(row[:2] == 0.0) and np.all(row[tgt] == 0.0) and np.all(row[25:] == 0.0)
+
+
 # ---------------------------------------------------------------------------------------
 # P3: strength 0 and neutral gains reduce to library attention (SDPA, fp64)
 # ---------------------------------------------------------------------------------------
