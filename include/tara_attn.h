@@ -225,9 +225,9 @@ int tara_quantize_qk_int8(const tara_tensor* Q, const tara_tensor* K, int8_t* q_
 
 /* Same operation, arguments and checks as tara_attn_forward for bf16/fp16 inputs, but it
  * never allocates: no cudaMalloc, no cudaFree, no allocating library call.  It is meant for
- * callers that cannot allocate device memory while they run (work recorded into CUDA graphs,
- * frameworks that own all device memory through their own pool, serving loops that must not
- * stall in the allocator).  The pages have no counterpart to this entry point.
+ * callers that cannot allocate device memory while they run (frameworks that own all device
+ * memory through their own pool, serving loops that must not stall in the allocator).  The
+ * pages have no counterpart to this entry point.
  *   - Scratch: a fixed module array of TARA_NOALLOC_SCRATCH_BYTES on each device instead of
  *     the cached workspace; sizes that need more return TARA_ERR_TOO_LARGE before anything
  *     is launched.  fp32 inputs return TARA_ERR_DTYPE (their kernel needs no scratch; call
@@ -238,7 +238,9 @@ int tara_quantize_qk_int8(const tara_tensor* Q, const tara_tensor* K, int8_t* q_
  *   - Sharing: every call on a device uses the same array and leaves its contents behind;
  *     calls never read what an earlier call left (each call rewrites every record it reads).
  *     Calls whose work overlaps on the GPU (different streams, or concurrent with each other)
- *     race on the array: serialise them on one stream.                                    */
+ *     race on the array: serialise them on one stream.
+ *   - Timing: a CUDA-event pair armed with tara_set_kernel_events brackets its attention
+ *     kernel, as for tara_attn_forward.                                                   */
 int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
                               const tara_token_meta* meta, const tara_params* p,
                               tara_tensor* O, float* LSE, void* stream);

@@ -16,7 +16,7 @@ Sources, by page and section:
     combine their log gains: binding k adds m_k * log(gain_k,i) for its own mask m_k.
   - "TARA: ...", "Three backends": the output is attention with its log-sum-exp.
 
-Readings taken where the pages are silent (each also listed in the design notes):
+Readings taken where the pages are silent:
   - per-token time is seconds on the shared, RoPE-aligned clock; a latent frame's tokens share
     one time; the time of frame f of a segment is t0 + f*frame_dt;
   - LSE is the natural-log log-sum-exp of the scaled, biased logits;

@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE (same restrictions as the rest of `oracle/`).
 
 "TARA: Native Temporal Alignment for MiniMax H3 References", section "Three backends": the
 one-pass kernels fuse the rule into dense INT8 attention.  The page does not give the scaling
-scheme; the reading taken here (also listed in the design notes):
+scheme; the reading taken here:
 
   - Q is quantised per token: each row of D values gets its own scale;
   - K is quantised per block of 128 consecutive tokens of one (branch, head): the block's

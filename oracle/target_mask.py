@@ -7,7 +7,7 @@
   - "Common issues": the mask must be one frame or exactly the prepared 17n+5 shot length
     (107 is such a length); any other length is an error.
 
-Readings where the page is silent (also listed in the design notes):
+Readings where the page is silent:
   - area downsampling is the exact area average: output cell (y, x) is the mean of the input
     over the rectangle [y*Hp/Hq, (y+1)*Hp/Hq) x [x*Wp/Wq, (x+1)*Wp/Wq) of the piecewise-
     constant input image (pixels straddling a cell boundary count by their overlap);

@@ -86,6 +86,59 @@ def _call(lib, Q=None, K=None, V=None, meta=None, p=None, O=None, lse=FAKE):
                                  ctypes.c_void_p(lse), None)
 
 
+def _call_noalloc(lib, Q, meta, p=None):
+    p = p if p is not None else B.make_params()
+    return lib.tara_attn_forward_noalloc(ctypes.byref(Q), ctypes.byref(Q), ctypes.byref(Q),
+                                         ctypes.byref(meta), ctypes.byref(p), ctypes.byref(Q),
+                                         ctypes.c_void_p(FAKE), None)
+
+
+def _noalloc_scratch(nsets, N):
+    """Bytes of scratch the allocation-free entry point needs: per metadata set a 32-byte
+    record per 128-token tile and a 16-byte record per token, each part rounded to 256."""
+    up = lambda x: (x + 255) // 256 * 256
+    return up(nsets * ((N + 127) // 128) * 32) + up(nsets * N * 16)
+
+
+def _noalloc_max_tokens(nsets):
+    cap = B.TARA_NOALLOC_SCRATCH_BYTES
+    N = cap // (16 * nsets)
+    while _noalloc_scratch(nsets, N) > cap:
+        N -= 1
+    return N
+
+
+@pytest.mark.parametrize("nsets", [1, 3])
+def test_noalloc_rejects_sizes_above_its_scratch(lib, nsets):
+    # one token more than the fixed array holds is refused before any CUDA call
+    header = open(os.path.join(ROOT, "include", "tara_attn.h")).read()
+    assert "#define TARA_NOALLOC_SCRATCH_BYTES (4u << 20)" in header
+    assert B.TARA_NOALLOC_SCRATCH_BYTES == 4 << 20
+    n_fit = _noalloc_max_tokens(nsets)
+    n = n_fit + 1
+    assert _noalloc_scratch(nsets, n) > B.TARA_NOALLOC_SCRATCH_BYTES
+    Q = _t(shape=(nsets, 2, n, 128))
+    m = _meta(N=n, stride=0 if nsets == 1 else n)
+    assert _call_noalloc(lib, Q, m) == -11   # TARA_ERR_TOO_LARGE
+    # its other refusals: fp32 inputs (no scratch needed) and 8-bit Q/K
+    assert _call_noalloc(lib, _t(dtype=B.TARA_FP32), _meta()) == -3
+    p = B.make_params()
+    p.qk_int8 = 1
+    assert _call_noalloc(lib, _t(), _meta(), p) == -5
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="a size that fits would launch on the fake pointers")
+@pytest.mark.parametrize("nsets", [1, 3])
+def test_noalloc_accepts_the_largest_size_that_fits(lib, nsets):
+    # the largest size passes the size check and stops at the first CUDA call (no device
+    # here), so the fake pointers are never used
+    n_fit = _noalloc_max_tokens(nsets)
+    Q = _t(shape=(nsets, 2, n_fit, 128))
+    m = _meta(N=n_fit, stride=0 if nsets == 1 else n_fit)
+    assert _call_noalloc(lib, Q, m) == -9   # TARA_ERR_CUDA
+
+
 def test_rejects_null(lib):
     assert lib.tara_attn_forward(None, None, None, None, None, None, None, None) == -1
     assert _call(lib, Q=_t(ptr=0)) == -1

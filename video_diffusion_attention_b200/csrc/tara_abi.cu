@@ -59,17 +59,20 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
 
+// Resolves the driver's tensor-map encoder once per process; both forward entry points call
+// this under different mutexes, so the lookup itself is guarded by its own once-flag.
 int get_encode_fn() {
-  if (g_encode) return TARA_OK;
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
-                                       &q) != cudaSuccess ||
-      q != cudaDriverEntryPointSuccess || fn == nullptr)
-    return TARA_ERR_CUDA;
-  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-  return TARA_OK;
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && fn != nullptr)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode ? TARA_OK : TARA_ERR_CUDA;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -566,10 +569,10 @@ int tara_device_status(void* stream_) {
 // ---------------------------------------------------------------------------------------
 // Allocation-free variant of the 16-bit forward pass.
 //
-// Some callers may not allocate device memory at call time: code that records work into a
-// CUDA graph or runs under a framework's own memory pool (cudaMalloc there either fails,
-// bypasses the pool's accounting, or synchronises the device in the middle of a step), and
-// latency-bound serving loops that must never hit the driver's allocator.  For them the
+// Some callers may not allocate device memory at call time: code that runs under a
+// framework's own memory pool (cudaMalloc there either fails, bypasses the pool's accounting,
+// or synchronises the device in the middle of a step), and latency-bound serving loops that
+// must never hit the driver's allocator.  For them the
 // scratch the tensor-core path needs (tile summaries and per-key bias records) lives in a
 // fixed device array that is part of the loaded module instead of the cached cudaMalloc
 // workspace used by tara_attn_forward.
@@ -621,8 +624,12 @@ int launch_tc_static(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
                            smem) != cudaSuccess)
     return TARA_ERR_CUDA;
   dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
+  // a kernel-event pair armed by tara_set_kernel_events times this launch, as in
+  // tara_attn_forward
+  if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
   attn_tc_kernel<kBF16, D><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, a);
-  return cudaGetLastError() == cudaSuccess ? TARA_OK : TARA_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
+  return record_stop(stream);
 }
 
 }  // namespace
