@@ -62,7 +62,7 @@ def load_peaks():
 
 
 # the device sources the attention kernel is compiled from
-KERNEL_SOURCES = ("attn_tc.cuh", "sm100_ptx.cuh", "tara_common.cuh")
+KERNEL_SOURCES = ("attn_pair.cuh", "attn_tc.cuh", "sm100_ptx.cuh", "tara_common.cuh")
 
 
 def kernel_source_hash() -> str:
@@ -76,6 +76,24 @@ def kernel_source_hash() -> str:
             code = "\n".join(line for line in lines if line)
         h.update(f.encode() + code.encode())
     return h.hexdigest()[:16]
+
+
+def clock_normalised(achieved: float, peak: float, kernel_mhz, peaks: dict) -> dict:
+    """The roofline fraction with the peak moved to the kernel's own SM clock.
+
+    The sustained peak was measured at the clock a dense GEMM settles at under the power cap;
+    a kernel that leaves the tensor pipe idle part of the time runs at a higher clock, which
+    flatters achieved/peak.  Scaling the peak by kernel MHz / peak MHz compares work per clock
+    cycle instead (the figure ncu's tensor-pipe-active counter reads).  None when either clock
+    is unknown."""
+    peak_mhz = (peaks.get("clocks_under_load") or {}).get("sm_mhz_median")
+    if not kernel_mhz or not peak_mhz:
+        return {"frac_at_kernel_clock": None, "kernel_sm_mhz_median": kernel_mhz,
+                "peak_sm_mhz_median": peak_mhz}
+    peak_at_clock = peak * float(kernel_mhz) / float(peak_mhz)
+    return {"frac_at_kernel_clock": achieved / peak_at_clock,
+            "peak_at_kernel_clock": peak_at_clock,
+            "kernel_sm_mhz_median": kernel_mhz, "peak_sm_mhz_median": peak_mhz}
 
 
 def recorded_traffic(workload: str):
@@ -431,6 +449,7 @@ def main():
         q8_line["roofline"] = {"bound": "tensor", "achieved": q8_ach, "peak": q8_peak,
                                "unit": "TFLOP/s", "frac": q8_ach / q8_peak,
                                "traffic": recorded_traffic(w.name + "_int8"),
+                               "clock_normalised": clock_normalised(q8_ach, q8_peak, clk.get("sm_mhz"), peaks),
                                "peak_kind": "QK^T at 2 x measured sustained bf16 (nominal int8 "
                                             "ratio), PV at measured sustained bf16 (%s)" % peak_src}
     if mask_line is not None:
@@ -451,7 +470,8 @@ def main():
             "nominal_2250": 100.0 * value / world / 2250.0, "peaks_source": peak_src},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "attn_tc_kernel", "kernel_ms": kmean,
+                     "kernel": "attn_pair_kernel", "kernel_ms": kmean,
+                     "clock_normalised": clock_normalised(achieved, peak, clk.get("sm_mhz"), peaks),
                      "kernel_ms_median": kernel_ms_median,
                      "peak_kind": "bf16_tflops_sustained (%s): the kernel runs back to back for "
                                   "seconds" % peak_src},

@@ -54,3 +54,16 @@ def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
     (src / bench.KERNEL_SOURCES[0]).write_text("int a = 1;\nint b = 3;\n")
     assert bench.kernel_source_hash() != h0
 
+
+
+def test_clock_normalised_fraction():
+    peaks = {"clocks_under_load": {"sm_mhz_median": 1300.0}}
+    # a kernel at twice the peak's clock: the per-clock fraction is half the plain one
+    r = bench.clock_normalised(1000.0, 1400.0, 2600.0, peaks)
+    assert abs(r["frac_at_kernel_clock"] - 1000.0 / 2800.0) < 1e-12
+    assert r["kernel_sm_mhz_median"] == 2600.0 and r["peak_sm_mhz_median"] == 1300.0
+    # at the peak's own clock both fractions agree
+    assert abs(bench.clock_normalised(700.0, 1400.0, 1300.0, peaks)["frac_at_kernel_clock"] - 0.5) < 1e-12
+    # an unknown clock gives no figure rather than a guess
+    assert bench.clock_normalised(1.0, 2.0, None, peaks)["frac_at_kernel_clock"] is None
+    assert bench.clock_normalised(1.0, 2.0, 1500.0, {})["frac_at_kernel_clock"] is None

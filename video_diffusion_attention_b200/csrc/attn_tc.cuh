@@ -133,6 +133,28 @@ __device__ __forceinline__ int row_max128_s32(const uint32_t (&s)[128]) {
   return max(max(max(a[0], a[1]), max(a[2], a[3])), max(max(a[4], a[5]), max(a[6], a[7])));
 }
 
+// Scores of one row of a per-edge (kClsFull) tile, in place: s[c] <- s[c]*sl + bias*log2(e),
+// with the bias of the edge (row, key c) from the staged key records kb (tara_common.cuh) and,
+// with chained bindings (kExtra), the row's weight wx[Picture index].  The bias is computed
+// for every row and zeroed by a select on non-target rows: a per-element branch on the row
+// role costs ~10x here.
+template <bool kExtra>
+__device__ __forceinline__ void add_edge_bias(uint32_t (&s)[128], const float4* kb, float t_q,
+                                              float m_q, bool is_tgt, float sl, const float* wx,
+                                              const BiasParams& bp) {
+  const float w = bp.window, inv_f = bp.inv_falloff, st = bp.strength, cap = bp.cap;
+#pragma unroll
+  for (int c = 0; c < 128; ++c) {
+    const float4 kv = kb[c];
+    const float x = fmaxf(fabsf(t_q - kv.x) - w, 0.0f) * inv_f;
+    const float pen = fminf(st * (x * x), cap);
+    float b = fmaf(-kv.z, pen, m_q * kv.y);
+    if (kExtra) b += wx[(int)kv.w];
+    b = is_tgt ? b : 0.0f;
+    s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl, b * kLog2e));
+  }
+}
+
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
   return kBF16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
@@ -427,30 +449,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       float mx, scl, off_base;
       if (cls == kClsFull) {
-        // branch-free per-edge bias: computed for every row, zeroed by a select on non-target
-        // rows (a per-element branch on the row role costs ~10x here)
-        const float w = bp.window, inv_f = bp.inv_falloff, st = bp.strength, cap = bp.cap;
-        if (bp.n_extra == 0) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const float4 kv = kb[c];
-            const float x = fmaxf(fabsf(t_q - kv.x) - w, 0.0f) * inv_f;
-            const float pen = fminf(st * (x * x), cap);
-            float b = fmaf(-kv.z, pen, m_q * kv.y);
-            b = is_tgt ? b : 0.0f;
-            s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl, b * kLog2e));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const float4 kv = kb[c];
-            const float x = fmaxf(fabsf(t_q - kv.x) - w, 0.0f) * inv_f;
-            const float pen = fminf(st * (x * x), cap);
-            float b = fmaf(-kv.z, pen, m_q * kv.y) + wx[(int)kv.w];
-            b = is_tgt ? b : 0.0f;
-            s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl, b * kLog2e));
-          }
-        }
+        if (bp.n_extra == 0) add_edge_bias<false>(s, kb, t_q, m_q, is_tgt, sl, wx, bp);
+        else add_edge_bias<true>(s, kb, t_q, m_q, is_tgt, sl, wx, bp);
         mx = row_max128(s);
         scl = 1.0f;
         off_base = 0.0f;

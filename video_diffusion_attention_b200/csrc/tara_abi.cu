@@ -11,6 +11,7 @@
 #include "tara_attn.h"
 #include "forward_internal.h"
 #include "param_checks.h"
+#include "attn_pair.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "quant_int8.cuh"
@@ -31,6 +32,7 @@ struct DeviceState {
   int* status = nullptr;        // device address of g_device_status
   bool tc_attr_set[2][2] = {{false, false}, {false, false}};   // [bf16][D==128]
   bool tc_q8_attr_set[2] = {false, false};                     // [bf16], D = 128
+  bool pair_attr_set[2] = {false, false};                      // [bf16], D = 128
   bool simt_attr_set = false;
   // recorded on a call's stream after its last workspace reader; the next call's stream waits
   // on it before rewriting the workspace, so calls on different streams serialise on the GPU
@@ -102,13 +104,15 @@ BiasParams make_bias_params(const tara_params* p, int D) {
   return bp;
 }
 
-int encode_qkv_map(CUtensorMap* map, const tara_tensor* t) {
+// Tensor map of a 16-bit [B*H][N][D] tensor: boxes of 64 head-dim columns (one 128-byte
+// swizzle panel) by box_rows tokens.
+int encode_qkv_map(CUtensorMap* map, const tara_tensor* t, uint32_t box_rows = kTile) {
   const CUtensorMapDataType dt =
       t->dtype == TARA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const cuuint64_t dims[3] = {(cuuint64_t)t->D, (cuuint64_t)t->N,
                               (cuuint64_t)t->B * (cuuint64_t)t->H};
   const cuuint64_t strides[2] = {(cuuint64_t)t->D * 2, (cuuint64_t)t->N * (cuuint64_t)t->D * 2};
-  const cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, dt, 3, t->ptr, dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -234,6 +238,31 @@ int launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& m
   dim3 grid((unsigned)((ntiles + 1) / 2), (unsigned)H, (unsigned)B);
   if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
   attn_tc_kernel<kBF16, D, kQ8><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, a);
+  if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
+  return record_stop(stream);
+}
+
+// Head dim 128, 16-bit Q/K: the SM-pair kernel.  Two CTAs per four query tiles; the K map
+// has 64-row boxes (each CTA of a pair loads half of every key tile).  `attr` caches the
+// one-time attribute set-up (nullptr: set it on every call).
+template <bool kBF16>
+int launch_pair(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
+                const TcArgs& a, int B, int H, int ntiles, cudaStream_t stream, bool* attr) {
+  constexpr int smem = PairShape::kSmemBytes;
+  if (!attr || !*attr) {
+    if (tc_register_check(attn_pair_kernel<kBF16>) != TARA_OK) return TARA_ERR_CUDA;
+    if (cudaFuncSetAttribute(attn_pair_kernel<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return TARA_ERR_CUDA;
+    if (attr) *attr = true;
+  }
+  CUtensorMap mq, mk, mv;
+  if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K, 64) != TARA_OK ||
+      encode_qkv_map(&mv, V) != TARA_OK)
+    return TARA_ERR_CUDA;
+  dim3 grid((unsigned)((ntiles + kPairTiles - 1) / kPairTiles * 2), (unsigned)H, (unsigned)B);
+  if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
+  attn_pair_kernel<kBF16><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, a);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
   return record_stop(stream);
 }
@@ -412,8 +441,8 @@ int forward_locked(const tara_tensor* Q, const tara_tensor* K, const tara_tensor
     rc = bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
               : launch_tc<false, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st);
   else if (D == 128)
-    rc = bf16 ? launch_tc<true, 128>(mq, mk, mv, a, B, H, ntiles, stream, st)
-              : launch_tc<false, 128>(mq, mk, mv, a, B, H, ntiles, stream, st);
+    rc = bf16 ? launch_pair<true>(Q, K, V, a, B, H, ntiles, stream, &st->pair_attr_set[1])
+              : launch_pair<false>(Q, K, V, a, B, H, ntiles, stream, &st->pair_attr_set[0]);
   else
     rc = bf16 ? launch_tc<true, 64>(mq, mk, mv, a, B, H, ntiles, stream, st)
               : launch_tc<false, 64>(mq, mk, mv, a, B, H, ntiles, stream, st);
@@ -675,8 +704,8 @@ extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor
       make_tc_args(meta, O, LSE, recs, keyinfo, N, H, ntiles, st->status, bp, nullptr, nullptr);
   const bool bf16 = Q->dtype == TARA_BF16;
   if (D == 128)
-    return bf16 ? launch_tc_static<true, 128>(mq, mk, mv, a, B, H, ntiles, stream)
-                : launch_tc_static<false, 128>(mq, mk, mv, a, B, H, ntiles, stream);
+    return bf16 ? launch_pair<true>(Q, K, V, a, B, H, ntiles, stream, nullptr)
+                : launch_pair<false>(Q, K, V, a, B, H, ntiles, stream, nullptr);
   return bf16 ? launch_tc_static<true, 64>(mq, mk, mv, a, B, H, ntiles, stream)
               : launch_tc_static<false, 64>(mq, mk, mv, a, B, H, ntiles, stream);
 }
