@@ -1,8 +1,13 @@
 // attn_pair.cuh -- the 16-bit, head-dim-128 tensor-core path on SM pairs, with P in shared
 // memory so that the next QK^T of a query tile does not wait for the previous PV.
 //
-// A cluster of two CTAs (an SM pair) owns four 128-row query tiles of one (branch, head): CTA r
-// of the pair holds tiles 4c + 2t + r for t = 0, 1.  The even CTA issues every MMA with
+// The kernel is persistent: one cluster of two CTAs (an SM pair) per two SMs, each walking work
+// items c, c + G, c + 2G, ... (G clusters) in head-major order.  An item is four 128-row query
+// tiles of one (branch, head): CTA r of the pair holds tiles 4q + 2t + r for t = 0, 1.  All
+// clusters start their n-th item at about the same time and stream the same head's K and V in
+// near lockstep, so a head's keys and values are read from DRAM about once and then served
+// from L2 to every cluster (a grid of one CTA pair per item let later waves re-read them).
+// The even CTA issues every MMA with
 // cta_group::2, M = 256: MMA "t" covers tile t of both CTAs.  Each CTA supplies its own 128 rows
 // of the A operand (Q for S = Q K^T, P for O += P V) and half of every B operand: keys
 // [64r, 64r + 64) of a key tile for QK^T and head-dim columns [64r, 64r + 64) of a value tile
@@ -51,7 +56,7 @@ struct PairShape {
   static constexpr int kPTileBytes = kTile * kTile * 2;   // 32 KB: P of one query tile
   static constexpr int kKeyBufBytes = 2 * 2 * kTile * 16; // [query tile][parity][key] float4
   static constexpr int kRowWBytes = 2 * kTile * 17 * 4;   // [tile][row] extra-binding weights
-  static constexpr int kBarCount = 1 + 2 * kStages + 2 * 4 + 2 + 1 + 2 + 8;
+  static constexpr int kBarCount = 2 + 2 * kStages + 2 * 4 + 2 + 1 + 2 + 8;
   static constexpr int kSmemBytes = 1024 /*alignment slack*/ + 2 * kQTileBytes +
                                     kStages * kHalfBytes + 2 * kPTileBytes + kKeyBufBytes +
                                     kRowWBytes + kBarCount * 8 + 16;
@@ -81,9 +86,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   float* rowx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(kbuf) + S::kKeyBufBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(rowx) + S::kRowWBytes);
   uint64_t* q_full = bars;              // even CTA: Q of both CTAs landed
-  uint64_t* kv_full = q_full + 1;       // even CTA: both halves of slot s landed
+  uint64_t* q_empty = q_full + 1;       // both CTAs (2-SM commit): the last QK^T of an item read Q
+  uint64_t* kv_full = q_empty + 1;      // even CTA: both halves of slot s landed
   uint64_t* kv_empty = kv_full + NS;    // both CTAs (2-SM commit): slot s may be refilled
-  uint64_t* s_full = kv_empty + NS;     // both CTAs (2-SM commit): S_t holds key tile j
+  uint64_t* s_full = kv_empty + NS;     // both CTAs (2-SM commit): S_t holds the next key tile
   uint64_t* s_free = s_full + 2;        // even CTA: 8 softmax warps have loaded S_t
   uint64_t* p_full = s_free + 2;        // even CTA: 8 softmax warps have stored P_t
   uint64_t* pv_done = p_full + 2;       // both CTAs (2-SM commit): PV_t completed
@@ -98,12 +104,19 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int N = args.N;
-  const int bh = blockIdx.z * args.H + blockIdx.y;
-  const int qt_base = (int)(blockIdx.x >> 1) * kPairTiles + (int)rank;   // + 2 t
   const int nk = (N + kTile - 1) / kTile;
+  // work items: (branch, head) planes x groups of four query tiles, head-major
+  const int groups = (args.ntiles + kPairTiles - 1) / kPairTiles;
+  const int n_items = args.B * args.H * groups;
+  const int n_clusters = (int)(gridDim.x >> 1);
+  const int first_item = (int)(blockIdx.x >> 1);
+  // Every role walks the same items in the same order.  Barrier phases run on across items:
+  // the g-th key tile this cluster processes (g = item ordinal * nk + j) completes phase g of
+  // the per-tile barriers, and ring slot s holds K or V half-tile number 2g or 2g + 1.
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -153,36 +166,47 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * S::kQTileBytes);
       const uint32_t q_full_l = mapa_shared(smem_u32(q_full), 0);
-      for (int t = 0; t < 2; ++t)
-        for (int p = 0; p < 2; ++p)
-          tma_load_3d_pair(sQ + t * S::kQTileBytes + p * S::kPanelBytes, &tmQ, q_full_l, p * 64,
-                           (qt_base + 2 * t) * kTile, bh);
+      // every cluster streams the same head's K and V at about the same time: keep them in L2;
+      // Q is read once per item
+      const uint64_t keep = l2_policy_evict_last(), once = l2_policy_evict_first();
+      bool ok = true;
+      int i = 0;   // half-tiles issued (K_j, V_j alternate)
       int issued = 0;
-      for (int i = 0; i < 2 * nk; ++i) {
-        const int slot = i % NS;
-        const uint32_t ph = (uint32_t)(i / NS) & 1u;
-        if (!mbar_wait(&kv_empty[slot], ph ^ 1u, abort_flag, kWaitLimitNs)) break;
-        if (leader) mbar_arrive_expect_tx(&kv_full[slot], 2 * HB);
-        const uint32_t full_l = mapa_shared(smem_u32(&kv_full[slot]), 0);
-        uint8_t* dst = sKV + slot * HB;
-        const int j = i >> 1;
-        if ((i & 1) == 0) {
-          // K_j rows [64r, 64r + 64): two 64-row x 128-byte panels (head-dim halves)
+      for (int item = first_item, k = 0; ok && item < n_items; item += n_clusters, ++k) {
+        const int bh = item / groups;
+        const int qt_base = (item - bh * groups) * kPairTiles + (int)rank;
+        // Q of the previous item is read by its last QK^T
+        if (k > 0 && !(ok = mbar_wait(q_empty, (uint32_t)(k - 1) & 1u, abort_flag, kWaitLimitNs))) break;
+        if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * S::kQTileBytes);
+        for (int t = 0; t < 2; ++t)
           for (int p = 0; p < 2; ++p)
-            tma_load_3d_pair(dst + p * (64 * 128), &tmK, full_l, p * 64,
-                             j * kTile + (int)rank * 64, bh);
-        } else {
-          // V_j head-dim columns [64r, 64r + 64): one 128-row x 128-byte panel
-          tma_load_3d_pair(dst, &tmV, full_l, (int)rank * 64, j * kTile, bh);
+            tma_load_3d_pair_hint(sQ + t * S::kQTileBytes + p * S::kPanelBytes, &tmQ, q_full_l,
+                                  p * 64, (qt_base + 2 * t) * kTile, bh, once);
+        for (int h2 = 0; h2 < 2 * nk; ++h2, ++i) {
+          const int slot = i % NS;
+          const uint32_t ph = (uint32_t)(i / NS) & 1u;
+          if (!(ok = mbar_wait(&kv_empty[slot], ph ^ 1u, abort_flag, kWaitLimitNs))) break;
+          if (leader) mbar_arrive_expect_tx(&kv_full[slot], 2 * HB);
+          const uint32_t full_l = mapa_shared(smem_u32(&kv_full[slot]), 0);
+          uint8_t* dst = sKV + slot * HB;
+          const int j = h2 >> 1;
+          if ((h2 & 1) == 0) {
+            // K_j rows [64r, 64r + 64): two 64-row x 128-byte panels (head-dim halves)
+            for (int p = 0; p < 2; ++p)
+              tma_load_3d_pair_hint(dst + p * (64 * 128), &tmK, full_l, p * 64,
+                                    j * kTile + (int)rank * 64, bh, keep);
+          } else {
+            // V_j head-dim columns [64r, 64r + 64): one 128-row x 128-byte panel
+            tma_load_3d_pair_hint(dst, &tmV, full_l, (int)rank * 64, j * kTile, bh, keep);
+          }
+          issued = i + 1;
         }
-        issued = i + 1;
       }
       if (*abort_flag && issued > 0) {
         // copies already issued land within microseconds; their completion is counted in the
         // even CTA, so give them 1 ms before this CTA's shared memory can be released
-        for (int k = 0; k < 1000; ++k) __nanosleep(1000);
+        for (int w = 0; w < 1000; ++w) __nanosleep(1000);
       }
     } else if ((warp == 9 || warp == 10) && lane == 0 && leader) {
       // ------------------------------ MMA issuers (even CTA) ---------------------------
@@ -198,55 +222,66 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // (shared addresses stay below 2^18, so the 14-bit field never carries)
         const uint64_t qd0 = make_sdesc_sw128(smem_u32(sQ), 16, 1024);
         const uint64_t kd0 = make_sdesc_sw128(smem_u32(sKV), 16, 1024);
-        ok = mbar_wait(q_full, 0, abort_flag, kWaitLimitNs);
-        for (int n = 0; ok && n < 2 * nk; ++n) {
-          const int t = n & 1, j = n >> 1;
-          const int ki = 2 * j, kslot = ki % NS;
-          // K_j is waited for once, for t = 0; its slot is released only after QK_1(j)
-          if (t == 0 && !(ok = mbar_wait(&kv_full[kslot], (uint32_t)(ki / NS) & 1u, abort_flag,
-                                         kWaitLimitNs)))
-            break;
-          // S_t is free once both CTAs' softmax warps have loaded key tile j-1 from it
-          if (j > 0 && !(ok = mbar_wait(&s_free[t], (uint32_t)(j - 1) & 1u, abort_flag,
-                                        kWaitLimitNs)))
-            break;
-          tc_fence_after();
-          const uint32_t d_s = tmem + (uint32_t)(t * 128);
-          const uint64_t qd = qd0 + (uint64_t)((t * S::kQTileBytes) >> 4);
-          const uint64_t kd = kd0 + (uint64_t)((kslot * HB) >> 4);
+        int g = 0;   // key tiles processed so far, over all items
+        for (int item = first_item, k = 0; ok && item < n_items; item += n_clusters, ++k) {
+          if (!(ok = mbar_wait(q_full, (uint32_t)k & 1u, abort_flag, kWaitLimitNs))) break;
+          for (int n = 0; ok && n < 2 * nk; ++n) {
+            const int t = n & 1, gj = g + (n >> 1);
+            const int ki = 2 * gj, kslot = ki % NS;
+            // K is waited for once, for t = 0; its slot is released only after QK_1
+            if (t == 0 && !(ok = mbar_wait(&kv_full[kslot], (uint32_t)(ki / NS) & 1u, abort_flag,
+                                           kWaitLimitNs)))
+              break;
+            // S_t is free once both CTAs' softmax warps have loaded the previous key tile
+            if (gj > 0 && !(ok = mbar_wait(&s_free[t], (uint32_t)(gj - 1) & 1u, abort_flag,
+                                           kWaitLimitNs)))
+              break;
+            tc_fence_after();
+            const uint32_t d_s = tmem + (uint32_t)(t * 128);
+            const uint64_t qd = qd0 + (uint64_t)((t * S::kQTileBytes) >> 4);
+            const uint64_t kd = kd0 + (uint64_t)((kslot * HB) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t qoff = (uint64_t)((((kk >> 2) * S::kPanelBytes) + (kk & 3) * 32) >> 4);
-            const uint64_t koff = (uint64_t)((((kk >> 2) * (64 * 128)) + (kk & 3) * 32) >> 4);
-            umma_ss_pair(d_s, qd + qoff, kd + koff, idesc_qk, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t qoff = (uint64_t)((((kk >> 2) * S::kPanelBytes) + (kk & 3) * 32) >> 4);
+              const uint64_t koff = (uint64_t)((((kk >> 2) * (64 * 128)) + (kk & 3) * 32) >> 4);
+              umma_ss_pair(d_s, qd + qoff, kd + koff, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit_pair(&s_full[t]);
+            if (t == 1) umma_commit_pair(&kv_empty[kslot]);
           }
-          umma_commit_pair(&s_full[t]);
-          if (t == 1) umma_commit_pair(&kv_empty[kslot]);
+          // the item's Q may be replaced once its last QK^T has read it
+          if (ok) umma_commit_pair(q_empty);
+          g += nk;
         }
       } else {
         constexpr uint32_t idesc_pv = make_idesc_f16(256, 128, kBF16, true);
         const uint64_t vd0 = make_sdesc_sw128(smem_u32(sKV), S::kPanelBytes, 1024);
         const uint64_t pd0 = make_sdesc_sw128(smem_u32(sP), 16, 1024);
-        for (int n = 0; ok && n < 2 * nk; ++n) {
-          const int t = n & 1, j = n >> 1;
-          const int vi = 2 * j + 1, vslot = vi % NS;
-          if (t == 0 && !(ok = mbar_wait(&kv_full[vslot], (uint32_t)(vi / NS) & 1u, abort_flag,
-                                         kWaitLimitNs)))
-            break;
-          // P_t(j) is in shared memory in both CTAs (and O_t rescaled where needed)
-          if (!(ok = mbar_wait(&p_full[t], (uint32_t)j & 1u, abort_flag, kWaitLimitNs))) break;
-          tc_fence_after();
-          const uint32_t d_o = tmem + S::kColO + (uint32_t)(t * 128);
-          const uint64_t pd = pd0 + (uint64_t)((t * S::kPTileBytes) >> 4);
-          const uint64_t vd = vd0 + (uint64_t)((vslot * HB) >> 4);
+        int g = 0;
+        for (int item = first_item; ok && item < n_items; item += n_clusters) {
+          for (int n = 0; ok && n < 2 * nk; ++n) {
+            const int t = n & 1, j = n >> 1, gj = g + j;
+            const int vi = 2 * gj + 1, vslot = vi % NS;
+            if (t == 0 && !(ok = mbar_wait(&kv_full[vslot], (uint32_t)(vi / NS) & 1u, abort_flag,
+                                           kWaitLimitNs)))
+              break;
+            // P_t is in shared memory in both CTAs (and O_t rescaled where needed)
+            if (!(ok = mbar_wait(&p_full[t], (uint32_t)gj & 1u, abort_flag, kWaitLimitNs))) break;
+            tc_fence_after();
+            const uint32_t d_o = tmem + S::kColO + (uint32_t)(t * 128);
+            const uint64_t pd = pd0 + (uint64_t)((t * S::kPTileBytes) >> 4);
+            const uint64_t vd = vd0 + (uint64_t)((vslot * HB) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t poff = (uint64_t)((((kk >> 2) * S::kPanelBytes) + (kk & 3) * 32) >> 4);
-            umma_ss_pair(d_o, pd + poff, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
-                         (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t poff = (uint64_t)((((kk >> 2) * S::kPanelBytes) + (kk & 3) * 32) >> 4);
+              // the first PV of an item starts O afresh
+              umma_ss_pair(d_o, pd + poff, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit_pair(&pv_done[t]);
+            if (t == 1) umma_commit_pair(&kv_empty[vslot]);
           }
-          umma_commit_pair(&pv_done[t]);
-          if (t == 1) umma_commit_pair(&kv_empty[vslot]);
+          g += nk;
         }
       }
       // every MMA this thread issued completes before either CTA releases its memory
@@ -261,206 +296,212 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int t = warp >> 2;            // query tile of this warpgroup
     const int wq = warp & 3;            // TMEM lane quarter
     const int r = wq * 32 + lane;       // row within the tile
-    const int qtile = qt_base + 2 * t;
-    const int row = qtile * kTile + r;
-    const bool row_ok = (qtile < args.ntiles) && (row < N);
     const BiasParams& bp = args.bp;
-    const int mset = args.per_branch_meta ? blockIdx.z : 0;
-    const long long mtok = (long long)mset * args.meta_stride;
-    const TileRec* recs = args.recs + (long long)mset * args.ntiles;
-    const float4* kinfo = args.keyinfo + (long long)mset * N;
     const uint32_t s_free_l = mapa_shared(smem_u32(&s_free[t]), 0);
     const uint32_t p_full_l = mapa_shared(smem_u32(&p_full[t]), 0);
     // this thread's row of P: 16-byte chunk c of panel p at p*16 KB + r*128 + ((c ^ (r%8))*16),
     // the 128-byte swizzle of a K-major operand (an 8-row atom of 1 KB per 8 rows)
     const uint32_t p_row = smem_u32(sP + t * S::kPTileBytes) + (uint32_t)(r * 128);
     const uint32_t p_sw = (uint32_t)(r & 7);
-
-    bool is_tgt = false;
-    float t_q = 0.0f, m_q = 0.0f;
-    if (row_ok) {
-      is_tgt = args.seg[mtok + row] == kSegTarget;
-      t_q = args.time_s[mtok + row];
-      m_q = args.m[mtok + row];
-    }
-    // weights of the extra bindings for this row, one per Picture index (0 for index 0)
-    float* wx = rowx + (t * kTile + r) * 17;
-    if (bp.n_extra > 0) {
-      for (int pidx = 0; pidx < 16; ++pidx) {
-        float acc = 0.0f;
-        if (is_tgt)
-          for (int k = 0; k < bp.n_extra; ++k)
-            acc += args.xm.m[k * args.xm.stride + mtok + row] * bp.lng_x[k][pidx];
-        wx[pidx] = acc;
-      }
-    }
-    TileRec qr;
-    if (qtile < args.ntiles) {
-      qr = recs[qtile];
-    } else {
-      qr.segmask = 0;
-      qr.picmask = 0;
-      qr.nvalid = 0;
-      qr.single_pic = 0;
-      qr.tq_min = qr.tk_min = 0.0f;
-      qr.tq_max = qr.tk_max = 0.0f;
-    }
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + (uint32_t)(t * 128);
     const uint32_t tO = tmem + lane_off + S::kColO + (uint32_t)(t * 128);
     const float ninf = __int_as_float(0xff800000);
-    float m_run = ninf, l_run = 0.0f;
+    // weights of the extra bindings for this row, one per Picture index (0 for index 0)
+    float* wx = rowx + (t * kTile + r) * 17;
     bool ok = true;
-
     uint32_t stage_phase = 0;
-    TileRec kr_next = recs[0];
-    for (int j = 0; j < nk; ++j) {
-      const TileRec kr = kr_next;
-      if (j + 1 < nk) kr_next = recs[j + 1];   // in flight while this tile is processed
-      const float sl = bp.scale_log2;
-      float cval;
-      const int cls = classify_pair(qr, kr, bp, &cval);
-      float rowb2 = 0.0f;
-      if (is_tgt) {
-        if (cls == kClsConstCap) rowb2 = cval * kLog2e;
-        else if (cls == kClsRowGuide) rowb2 = -penalty_f32(fabsf(t_q - kr.tk_min), bp) * kLog2e;
-        else if (cls == kClsConstPic)
-          rowb2 = (bp.n_extra > 0 ? m_q * cval + wx[kr.single_pic & 15] : m_q * cval) * kLog2e;
-      }
-      float4* kb = kbuf + (t * 2 + (j & 1)) * kTile;
-      if (cls == kClsFull) {
-        // stage the tile's key records in shared memory (one coalesced load per thread); two
-        // buffers, so a warp one iteration ahead never overwrites records another warp of the
-        // group still reads
-        const int key = j * kTile + r;
-        kb[r] = key < N ? kinfo[key] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        if (!(ok = warp_rendezvous(&stage_bar[t], stage_phase, abort_flag, kWaitLimitNs))) break;
-      }
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], (uint32_t)j & 1u,
-                                                           abort_flag, kWaitLimitNs))))
-        break;
-      tc_fence_after();
-      uint32_t s[128];
-      tmem_ld128(tS, s);
-      tmem_ld_wait();
-      reg_fence<128>(s);
-      // S_t may now be overwritten by the next key tile's QK^T
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(s_free_l);
+    int g = 0;   // key tiles processed so far, over all items
 
-      const int nv = (int)kr.nvalid;
-      if (nv < kTile) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= nv) s[c] = 0xff800000u;
+    for (int item = first_item; ok && item < n_items; item += n_clusters, g += nk) {
+      const int bh = item / groups;
+      const int qtile = (item - bh * groups) * kPairTiles + (int)rank + 2 * t;
+      const int row = qtile * kTile + r;
+      const bool row_ok = (qtile < args.ntiles) && (row < N);
+      const int mset = args.per_branch_meta ? bh / args.H : 0;
+      const long long mtok = (long long)mset * args.meta_stride;
+      const TileRec* recs = args.recs + (long long)mset * args.ntiles;
+      const float4* kinfo = args.keyinfo + (long long)mset * N;
+
+      bool is_tgt = false;
+      float t_q = 0.0f, m_q = 0.0f;
+      if (row_ok) {
+        is_tgt = args.seg[mtok + row] == kSegTarget;
+        t_q = args.time_s[mtok + row];
+        m_q = args.m[mtok + row];
       }
-      float mx, scl, off_base;
-      if (cls == kClsFull) {
-        if (bp.n_extra == 0) add_edge_bias<false>(s, kb, t_q, m_q, is_tgt, sl, wx, bp);
-        else add_edge_bias<true>(s, kb, t_q, m_q, is_tgt, sl, wx, bp);
-        mx = row_max128(s);
-        scl = 1.0f;
-        off_base = 0.0f;
+      if (bp.n_extra > 0) {
+        for (int pidx = 0; pidx < 16; ++pidx) {
+          float acc = 0.0f;
+          if (is_tgt)
+            for (int kx = 0; kx < bp.n_extra; ++kx)
+              acc += args.xm.m[kx * args.xm.stride + mtok + row] * bp.lng_x[kx][pidx];
+          wx[pidx] = acc;
+        }
+      }
+      TileRec qr;
+      if (qtile < args.ntiles) {
+        qr = recs[qtile];
       } else {
-        mx = fmaf(row_max128(s), sl, rowb2);
-        scl = sl;
-        off_base = rowb2;
+        qr.segmask = 0;
+        qr.picmask = 0;
+        qr.nvalid = 0;
+        qr.single_pic = 0;
+        qr.tq_min = qr.tk_min = 0.0f;
+        qr.tq_max = qr.tk_max = 0.0f;
       }
-      const float m_new = fmaxf(m_run, mx);
-      const bool need = (m_new - m_run) > 8.0f;        // true on the first tile (m_run = -inf)
-      const bool warp_need = __any_sync(0xffffffffu, need);
-      const float m_use = need ? m_new : m_run;
-      const float alpha = ex2_approx(m_run - m_use);   // 1 when not raised, 0 on the first tile
-      l_run *= alpha;
-      const float off = off_base - m_use;
-      // The two warps of a lane quarter (one per query tile) share an SM sub-partition and its
-      // exponential unit, which both tiles together keep busy for as long as the tensor pipe
-      // needs per key tile.  Their exponential phases take turns (tile 0 of key tile j, tile 1
-      // of j, tile 0 of j+1, ...), so that one warp's loads, max and stores overlap the other's
-      // exponentials instead of both warps contending for the unit at once.
-      if (!(ok = warp_wait(&exp_tok[2 * wq + t], (uint32_t)j & 1u, abort_flag, kWaitLimitNs))) break;
-      // all 128 exponentials first, into 64 packed 16-bit pairs (each score register dies as
-      // its pair is formed); columns in pairs: one packed FMA forms both exponents, one packed
-      // add accumulates both probabilities (two accumulators break the dependency chain)
-      const uint64_t scl2 = f32x2_pack(scl, scl), off2 = f32x2_pack(off, off);
-      uint64_t lsum2[2] = {0ull, 0ull};
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        float x0, x1;
-        f32x2_unpack(f32x2_fma(f32x2_pack_bits(s[c], s[c + 1]), scl2, off2), x0, x1);
-        const float p0 = ex2_approx(x0);
-        const float p1 = ex2_approx(x1);
-        lsum2[(c >> 1) & 1] = f32x2_add(lsum2[(c >> 1) & 1], f32x2_pack(p0, p1));
-        pk[c >> 1] = pack_p<kBF16>(p0, p1);
-      }
-      {
-        float a0, a1;
-        f32x2_unpack(f32x2_add(lsum2[0], lsum2[1]), a0, a1);
-        l_run += a0 + a1;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&exp_tok[2 * wq + (t ^ 1)]);
-      // the P buffer's previous reader (and the last writer of O_t) is PV_t(j-1)
-      if (j > 0) {
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[t], (uint32_t)(j - 1) & 1u,
-                                                             abort_flag, kWaitLimitNs))))
-          break;
+      float m_run = ninf, l_run = 0.0f;
+
+      TileRec kr_next = recs[0];
+      for (int j = 0; j < nk; ++j) {
+        const int gj = g + j;
+        const TileRec kr = kr_next;
+        if (j + 1 < nk) kr_next = recs[j + 1];   // in flight while this tile is processed
+        const float sl = bp.scale_log2;
+        float cval;
+        const int cls = classify_pair(qr, kr, bp, &cval);
+        float rowb2 = 0.0f;
+        if (is_tgt) {
+          if (cls == kClsConstCap) rowb2 = cval * kLog2e;
+          else if (cls == kClsRowGuide) rowb2 = -penalty_f32(fabsf(t_q - kr.tk_min), bp) * kLog2e;
+          else if (cls == kClsConstPic)
+            rowb2 = (bp.n_extra > 0 ? m_q * cval + wx[kr.single_pic & 15] : m_q * cval) * kLog2e;
+        }
+        float4* kb = kbuf + (t * 2 + (gj & 1)) * kTile;
+        if (cls == kClsFull) {
+          // stage the tile's key records in shared memory (one coalesced load per thread);
+          // two buffers, so a warp one iteration ahead never overwrites records another warp
+          // of the group still reads
+          const int key = j * kTile + r;
+          kb[r] = key < N ? kinfo[key] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (!(ok = warp_rendezvous(&stage_bar[t], stage_phase, abort_flag, kWaitLimitNs))) break;
+        }
+        if (!(ok = warp_wait(&s_full[t], (uint32_t)gj & 1u, abort_flag, kWaitLimitNs))) break;
         tc_fence_after();
-      }
+        uint32_t s[128];
+        tmem_ld128(tS, s);
+        tmem_ld_wait();
+        reg_fence<128>(s);
+        // S_t may now be overwritten by the next key tile's QK^T
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(s_free_l);
+
+        const int nv = (int)kr.nvalid;
+        if (nv < kTile) {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint32_t addr = p_row + (uint32_t)((c >> 3) * S::kPanelBytes) +
-                              ((((uint32_t)c & 7u) ^ p_sw) << 4);
-        st_shared_v4(addr, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c = 0; c < 128; ++c)
+            if (c >= nv) s[c] = 0xff800000u;
+        }
+        float mx, scl, off_base;
+        if (cls == kClsFull) {
+          if (bp.n_extra == 0) add_edge_bias<false>(s, kb, t_q, m_q, is_tgt, sl, wx, bp);
+          else add_edge_bias<true>(s, kb, t_q, m_q, is_tgt, sl, wx, bp);
+          mx = row_max128(s);
+          scl = 1.0f;
+          off_base = 0.0f;
+        } else {
+          mx = fmaf(row_max128(s), sl, rowb2);
+          scl = sl;
+          off_base = rowb2;
+        }
+        const float m_new = fmaxf(m_run, mx);
+        const bool need = (m_new - m_run) > 8.0f;        // true on the first tile (m_run = -inf)
+        const bool warp_need = __any_sync(0xffffffffu, need);
+        const float m_use = need ? m_new : m_run;
+        const float alpha = ex2_approx(m_run - m_use);   // 1 when not raised, 0 on the first tile
+        l_run *= alpha;
+        const float off = off_base - m_use;
+        // The two warps of a lane quarter (one per query tile) share an SM sub-partition and
+        // its exponential unit, which both tiles together keep busy for as long as the tensor
+        // pipe needs per key tile.  Their exponential phases take turns (tile 0 of one key
+        // tile, tile 1 of it, tile 0 of the next, ...), so that one warp's loads, max and
+        // stores overlap the other's exponentials instead of both contending for the unit.
+        if (!(ok = warp_wait(&exp_tok[2 * wq + t], (uint32_t)gj & 1u, abort_flag, kWaitLimitNs))) break;
+        // all 128 exponentials first, into 64 packed 16-bit pairs (each score register dies as
+        // its pair is formed); columns in pairs: one packed FMA forms both exponents, one
+        // packed add accumulates both probabilities (two accumulators break the dependency
+        // chain)
+        const uint64_t scl2 = f32x2_pack(scl, scl), off2 = f32x2_pack(off, off);
+        uint64_t lsum2[2] = {0ull, 0ull};
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          float x0, x1;
+          f32x2_unpack(f32x2_fma(f32x2_pack_bits(s[c], s[c + 1]), scl2, off2), x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          lsum2[(c >> 1) & 1] = f32x2_add(lsum2[(c >> 1) & 1], f32x2_pack(p0, p1));
+          pk[c >> 1] = pack_p<kBF16>(p0, p1);
+        }
+        {
+          float a0, a1;
+          f32x2_unpack(f32x2_add(lsum2[0], lsum2[1]), a0, a1);
+          l_run += a0 + a1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&exp_tok[2 * wq + (t ^ 1)]);
+        // the P buffer's previous reader (and the last writer of O_t) is the previous PV_t
+        if (gj > 0) {
+          if (!(ok = warp_wait(&pv_done[t], (uint32_t)(gj - 1) & 1u, abort_flag, kWaitLimitNs))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint32_t addr = p_row + (uint32_t)((c >> 3) * S::kPanelBytes) +
+                                ((((uint32_t)c & 7u) ^ p_sw) << 4);
+          st_shared_v4(addr, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        if (j > 0 && warp_need) {
+          // rescale this warp's O rows; the previous PV_t has landed and the next waits for P
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_ld_wait();
+            reg_fence<32>(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(tO + cc * 32, o);
+          }
+          tmem_st_wait();
+        }
+        m_run = m_use;
+        // P (generic-proxy stores) must be visible to the tensor core (async proxy)
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(p_full_l);
       }
-      if (j > 0 && warp_need) {
-        // rescale this warp's O rows; PV_t(j-1) has landed and PV_t(j) waits for P_t(j)
+
+      // ------------------------------ epilogue of the item ---------------------------
+      // The next item's first PV_t overwrites O_t; it waits for this warp's P of that item,
+      // which comes after these reads in program order.
+      if (ok && (ok = warp_wait(&pv_done[t], (uint32_t)(g + nk - 1) & 1u, abort_flag, kWaitLimitNs))) {
+        tc_fence_after();
+        const float inv_l = 1.0f / l_run;
+        uint16_t* orow = reinterpret_cast<uint16_t*>(args.O) + ((long long)bh * N + row) * D;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(tO + cc * 32, o);
           tmem_ld_wait();
           reg_fence<32>(o);
+          if (row_ok) {
+            uint32_t w[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(tO + cc * 32, o);
+            for (int c = 0; c < 16; ++c)
+              w[c] = pack_p<kBF16>(__uint_as_float(o[2 * c]) * inv_l,
+                                   __uint_as_float(o[2 * c + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              st_global_v4_stream(dst + v, make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]));
+          }
         }
-        tmem_st_wait();
+        if (row_ok) args.LSE[(long long)bh * N + row] = (m_run + log2f(l_run)) * kLn2;
+        tc_fence_before();
       }
-      m_run = m_use;
-      // P (generic-proxy stores) must be visible to the tensor core (async proxy)
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(p_full_l);
-    }
-
-    // ------------------------------ epilogue ---------------------------------------
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&pv_done[t], (uint32_t)(nk - 1) & 1u,
-                                                        abort_flag, kWaitLimitNs))) {
-      tc_fence_after();
-      const float inv_l = 1.0f / l_run;
-      uint16_t* orow = reinterpret_cast<uint16_t*>(args.O) + ((long long)bh * N + row) * D;
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_ld_wait();
-        reg_fence<32>(o);
-        if (row_ok) {
-          uint32_t w[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            w[c] = pack_p<kBF16>(__uint_as_float(o[2 * c]) * inv_l,
-                                 __uint_as_float(o[2 * c + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-        }
-      }
-      if (row_ok) args.LSE[(long long)bh * N + row] = (m_run + log2f(l_run)) * kLn2;
     }
     tc_fence_before();
   }

@@ -79,6 +79,7 @@ struct TcArgs {
   const float4* keyinfo;
   long long meta_stride;   // tokens between metadata sets (0: one set for all branches)
   int N, H, ntiles;
+  int B;                   // branches (the persistent kernel walks all B x H planes)
   int per_branch_meta;     // 1 when every branch has its own metadata set
   int* status;
   BiasParams bp;

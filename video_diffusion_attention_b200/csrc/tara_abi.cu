@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -260,7 +261,15 @@ int launch_pair(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V
   if (encode_qkv_map(&mq, Q) != TARA_OK || encode_qkv_map(&mk, K, 64) != TARA_OK ||
       encode_qkv_map(&mv, V) != TARA_OK)
     return TARA_ERR_CUDA;
-  dim3 grid((unsigned)((ntiles + kPairTiles - 1) / kPairTiles * 2), (unsigned)H, (unsigned)B);
+  // persistent: one cluster per SM pair (at most one per work item), each walking the
+  // (branch, head, 4-query-tile) items in head-major order
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return TARA_ERR_CUDA;
+  const long long items = (long long)B * H * ((ntiles + kPairTiles - 1) / kPairTiles);
+  const long long clusters = std::min<long long>(items, std::max(1, sms / 2));
+  dim3 grid((unsigned)(2 * clusters), 1, 1);
   if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
   attn_pair_kernel<kBF16><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, a);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
@@ -283,6 +292,7 @@ TcArgs make_tc_args(const tara_token_meta* meta, tara_tensor* O, float* LSE, Til
   a.N = N;
   a.H = H;
   a.ntiles = ntiles;
+  a.B = O->B;
   a.per_branch_meta = meta->batch_stride != 0 ? 1 : 0;
   a.status = status;
   a.bp = bp;
