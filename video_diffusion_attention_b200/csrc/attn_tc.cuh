@@ -124,14 +124,21 @@ __device__ __forceinline__ bool warp_rendezvous(uint64_t* bar, uint32_t& phase,
   return ok;
 }
 
-// Max of 128 signed 32-bit values (the 8-bit path's integer scores).
+// Max of 128 signed 32-bit values (the 8-bit path's integer scores): eight independent
+// chains of three-input integer max, then a tree (64 operations instead of 127).
 __device__ __forceinline__ int row_max128_s32(const uint32_t (&s)[128]) {
   int a[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) a[i] = (int)s[i];
 #pragma unroll
-  for (int c = 8; c < 128; ++c) a[c & 7] = max(a[c & 7], (int)s[c]);
-  return max(max(max(a[0], a[1]), max(a[2], a[3])), max(max(a[4], a[5]), max(a[6], a[7])));
+  for (int c = 8; c < 120; c += 16) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = __vimax3_s32(a[i], (int)s[c + i], (int)s[c + 8 + i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = max(a[i], (int)s[120 + i]);
+  return __vimax3_s32(__vimax3_s32(a[0], a[1], a[2]), __vimax3_s32(a[3], a[4], a[5]),
+                      max(a[6], a[7]));
 }
 
 // Scores of one row of a per-edge (kClsFull) tile, in place: s[c] <- s[c]*sl + bias*log2(e),
