@@ -67,6 +67,7 @@ extern "C" {
 #define TARA_ERR_DEVICE_TIMEOUT -10  /* a kernel gave up on a bounded wait (see below)      */
 #define TARA_ERR_TOO_LARGE      -11  /* a size exceeds what an index type or buffer holds   */
 #define TARA_ERR_MASK_LENGTH    -12  /* mask neither one frame nor the 17n+5 shot length    */
+#define TARA_ERR_DEBUG_CHECK    -13  /* debug build: a device-side check failed (see below)  */
 
 /* ---- token roles ---------------------------------------------------------------------- */
 /* Roles of the tokens of the packed joint sequence ("TARA: ...", opening paragraphs and
@@ -258,6 +259,16 @@ int tara_set_kernel_events(void* start, void* stop);
  * `stream`, returns TARA_ERR_DEVICE_TIMEOUT if the word is set (and clears it), TARA_ERR_CUDA
  * if the synchronisation failed, TARA_OK otherwise.                                       */
 int tara_device_status(void* stream);
+
+/* Debug build.  The library can be compiled with -DTARA_DEBUG=1 (python -m
+ * video_diffusion_attention_b200.build --debug writes libtara_attn_debug.so beside the release
+ * library).  Its kernels then check on the device what the host cannot see: that target and
+ * guide tokens carry finite times and target tokens finite mask weights, and that every row,
+ * plane and output index they derive stays inside its array.  A failed check records itself
+ * in the status word, the checked access is skipped and nothing traps; tara_device_status
+ * then returns TARA_ERR_DEBUG_CHECK (and clears the word).  The release build has no such
+ * checks.  Returns 1 in the debug build, 0 otherwise.  The pages have no counterpart.     */
+int tara_debug_build(void);
 
 /* Self-test of that machinery (failure detection without faulting the GPU): launches one
  * warp on `stream` that waits on a shared-memory barrier with a limit of limit_us

@@ -43,6 +43,14 @@ def test_library_exports_every_declared_function(lib):
     assert set(B.EXPORTS) <= names
 
 
+def test_debug_build_flag(lib):
+    # the release library has no device-side checks; its debug twin compiles them in
+    assert lib.tara_debug_build() == 0
+    dbg = B.load_library(libbuild.build(debug=True))
+    assert dbg.tara_debug_build() == 1
+    assert b"debug" in lib.tara_status_string(-13)
+
+
 def test_status_strings(lib):
     for code in list(B.STATUS) + [-99]:
         assert lib.tara_status_string(code)

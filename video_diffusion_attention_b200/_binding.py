@@ -25,11 +25,13 @@ STATUS = {
     -4: "TARA_ERR_HEAD_DIM", -5: "TARA_ERR_PARAM", -6: "TARA_ERR_ALIGN",
     -7: "TARA_ERR_SEGMENT", -8: "TARA_ERR_CAPACITY", -9: "TARA_ERR_CUDA",
     -10: "TARA_ERR_DEVICE_TIMEOUT", -11: "TARA_ERR_TOO_LARGE", -12: "TARA_ERR_MASK_LENGTH",
+    -13: "TARA_ERR_DEBUG_CHECK",
 }
 EXPORTS = ("tara_default_params", "tara_status_string", "tara_attn_forward",
            "tara_device_status", "tara_packed_length", "tara_pack_token_meta",
            "tara_set_kernel_events", "tara_selftest_wait", "tara_attn_forward_noalloc",
-           "tara_prepare_target_mask", "tara_quantize_qk_int8", "tara_attn_forward_host")
+           "tara_prepare_target_mask", "tara_quantize_qk_int8", "tara_attn_forward_host",
+           "tara_debug_build")
 
 
 class TaraError(RuntimeError):
@@ -105,6 +107,8 @@ def load_library(path: Optional[str] = None):
     lib.tara_selftest_wait.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
     lib.tara_device_status.restype = ctypes.c_int
     lib.tara_device_status.argtypes = [ctypes.c_void_p]
+    lib.tara_debug_build.restype = ctypes.c_int
+    lib.tara_debug_build.argtypes = []
     lib.tara_packed_length.restype = ctypes.c_int64
     lib.tara_packed_length.argtypes = [ctypes.POINTER(TaraSegment), ctypes.c_int32]
     lib.tara_pack_token_meta.restype = ctypes.c_int

@@ -13,6 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libtara_attn.so")
+# the same sources with the kernels' device-side checks compiled in (-DTARA_DEBUG=1)
+LIB_DEBUG = os.path.join(LIB_DIR, "libtara_attn_debug.so")
 SOURCES = [os.path.join(CSRC, "tara_abi.cu"), os.path.join(CSRC, "tara_pack.cpp"),
            os.path.join(CSRC, "tara_host.cpp")]
 HEADERS = [os.path.join(ROOT, "include", "tara_attn.h")] + [
@@ -32,26 +34,32 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in SOURCES + HEADERS)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not stale():
-        return LIB
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    """Compile the release library (or, with debug=True, libtara_attn_debug.so with the
+    kernels' device-side checks) if a source is newer than it or force is set."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not stale(lib):
+        return lib
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB + ".tmp%d" % os.getpid()
+    tmp = lib + ".tmp%d" % os.getpid()
     cmd = [nvcc()] + NVCC_FLAGS + ["-I", os.path.join(ROOT, "include"), "-I", CSRC]
+    if debug:
+        cmd += ["-DTARA_DEBUG=1"]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     cmd += ["-o", tmp] + SOURCES
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv))
+    print(build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv,
+                debug="--debug" in sys.argv))

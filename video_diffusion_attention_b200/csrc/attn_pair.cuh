@@ -330,6 +330,12 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         t_q = args.time_s[mtok + row];
         m_q = args.m[mtok + row];
       }
+      // debug build: the plane exists, a target row's time and mask weight are finite, and
+      // this row's part of P stays inside its tile's buffer
+      TARA_DCHECK_RECORD(bh < args.B * args.H, args.status);
+      TARA_DCHECK_RECORD(!is_tgt || (isfinite(t_q) && isfinite(m_q)), args.status);
+      TARA_DCHECK_RECORD(p_row + S::kPanelBytes + 128 <= smem_u32(sP) + (uint32_t)(t + 1) * S::kPTileBytes,
+                  args.status);
       if (bp.n_extra > 0) {
         for (int pidx = 0; pidx < 16; ++pidx) {
           float acc = 0.0f;
@@ -481,13 +487,15 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tc_fence_after();
         const float inv_l = 1.0f / l_run;
         uint16_t* orow = reinterpret_cast<uint16_t*>(args.O) + ((long long)bh * N + row) * D;
+        const bool out_ok =
+            row_ok && TARA_DCHECK((long long)bh * N + row < (long long)args.B * args.H * N, args.status);
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(tO + cc * 32, o);
           tmem_ld_wait();
           reg_fence<32>(o);
-          if (row_ok) {
+          if (out_ok) {
             uint32_t w[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c)
@@ -499,7 +507,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
               st_global_v4_stream(dst + v, make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]));
           }
         }
-        if (row_ok) args.LSE[(long long)bh * N + row] = (m_run + log2f(l_run)) * kLn2;
+        if (out_ok) args.LSE[(long long)bh * N + row] = (m_run + log2f(l_run)) * kLn2;
         tc_fence_before();
       }
     }

@@ -19,7 +19,8 @@ attn_simt_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                  const float* __restrict__ V, float* __restrict__ O, float* __restrict__ LSE,
                  const uint8_t* __restrict__ seg, const float* __restrict__ time_s,
                  const uint8_t* __restrict__ pic, const float* __restrict__ mw,
-                 long long batch_stride, int H, int N, int D, BiasParams bp, ExtraMasks xm) {
+                 long long batch_stride, int H, int N, int D, BiasParams bp, ExtraMasks xm,
+                 int* status) {
   extern __shared__ float smem[];
   const int ld = D + 1;                           // padded row: conflict-free column reads
   float* sK = smem;                               // [chunk][ld]
@@ -38,6 +39,8 @@ attn_simt_kernel(const float* __restrict__ Q, const float* __restrict__ K,
   const bool tgt = row_ok && seg[mb + row] == kSegTarget;
   const float t_q = row_ok ? time_s[mb + row] : 0.0f;
   const float m_q = row_ok ? mw[mb + row] : 0.0f;
+  // debug build: a target row's time and mask weight are finite numbers
+  if (lane == 0) TARA_DCHECK_RECORD(!tgt || (isfinite(t_q) && isfinite(m_q)), status);
 
   const float ninf = __int_as_float(0xff800000);
   float m_run = ninf, l_run = 0.0f;

@@ -366,6 +366,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       t_q = args.time_s[mtok + row];
       m_q = args.m[mtok + row];
     }
+    // debug build: the plane exists and a target row's time and mask weight are finite
+    TARA_DCHECK_RECORD(bh < args.B * args.H, args.status);
+    TARA_DCHECK_RECORD(!is_tgt || (isfinite(t_q) && isfinite(m_q)), args.status);
     // logit scale in log2 units; with 8-bit Q/K it also carries the row's and the key tile's
     // dequantisation scales
     const float row_sl = kQ8 ? bp.scale_log2 * (row_ok ? args.q_scale[(long long)bh * N + row] : 0.0f)
@@ -530,13 +533,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
       uint16_t* orow = reinterpret_cast<uint16_t*>(args.O) + ((long long)bh * N + row) * D;
+      const bool out_ok =
+          row_ok && TARA_DCHECK((long long)bh * N + row < (long long)args.B * args.H * N, args.status);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
         tmem_ld32(tO + cc * 32, o);
         tmem_ld_wait();
         reg_fence<32>(o);
-        if (row_ok) {
+        if (out_ok) {
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c)
@@ -547,7 +552,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
-      if (row_ok) args.LSE[(long long)bh * N + row] = (m_run + log2f(l_run)) * kLn2;
+      if (out_ok) args.LSE[(long long)bh * N + row] = (m_run + log2f(l_run)) * kLn2;
     }
     tc_fence_before();
   }

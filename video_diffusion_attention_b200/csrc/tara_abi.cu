@@ -397,7 +397,7 @@ int forward_locked(const tara_tensor* Q, const tara_tensor* K, const tara_tensor
         static_cast<const float*>(Q->ptr), static_cast<const float*>(K->ptr),
         static_cast<const float*>(V->ptr), static_cast<float*>(O->ptr), LSE, meta->seg,
         meta->time_s, meta->pic, meta->m, (long long)meta->batch_stride, H, N, D, bp,
-        ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride});
+        ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride}, st->status);
     if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
     return record_stop(stream);
   }
@@ -442,7 +442,7 @@ int forward_locked(const tara_tensor* Q, const tara_tensor* K, const tara_tensor
 
   tile_summary_kernel<<<dim3((unsigned)ntiles, (unsigned)L.nsets), 128, 0, stream>>>(
       meta->seg, meta->time_s, meta->pic, N, (long long)meta->batch_stride, ntiles, bp, recs,
-      keyinfo);
+      keyinfo, st->status);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
 
   const TcArgs a = make_tc_args(meta, O, LSE, recs, keyinfo, N, H, ntiles, st->status, bp, qs, ks);
@@ -514,6 +514,7 @@ const char* tara_status_string(int s) {
     case TARA_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
     case TARA_ERR_TOO_LARGE: return "size too large";
     case TARA_ERR_MASK_LENGTH: return "mask is neither one frame nor the prepared shot length";
+    case TARA_ERR_DEBUG_CHECK: return "a device-side check of the debug build failed";
     default: return "unknown status";
   }
 }
@@ -598,12 +599,21 @@ int tara_device_status(void* stream_) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return TARA_ERR_CUDA;
-    return TARA_ERR_DEVICE_TIMEOUT;
+    // bit 1: a device-side check of the debug build failed; bit 0: a bounded wait gave up
+    return (v & 2) ? TARA_ERR_DEBUG_CHECK : TARA_ERR_DEVICE_TIMEOUT;
   }
   return TARA_OK;
 }
 
 }  // extern "C"
+
+extern "C" int tara_debug_build(void) {
+#if defined(TARA_DEBUG) && TARA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 // ---------------------------------------------------------------------------------------
 // Allocation-free variant of the 16-bit forward pass.
@@ -707,7 +717,7 @@ extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor
   // clearing between calls
   tile_summary_kernel<<<dim3((unsigned)ntiles, (unsigned)nsets), 128, 0, stream>>>(
       meta->seg, meta->time_s, meta->pic, N, (long long)meta->batch_stride, ntiles, bp, recs,
-      keyinfo);
+      keyinfo, st->status);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
 
   const TcArgs a =

@@ -11,6 +11,22 @@ constexpr float kLog2e = 1.4426950408889634f;   // log2(e)
 constexpr float kLn2 = 0.6931471805599453f;     // ln(2)
 constexpr int kTile = 128;                       // tokens per tile (rows and keys)
 
+// Device-side checks of the debug build (compiled with -DTARA_DEBUG=1): a failed check sets
+// bit 1 of the device status word (tara_device_status then reports TARA_ERR_DEBUG_CHECK);
+// nothing traps.  TARA_DCHECK is an expression that guards an access (the access is skipped
+// when the check fails), TARA_DCHECK_RECORD a statement that only records.  The release
+// build evaluates neither condition.
+#if defined(TARA_DEBUG) && TARA_DEBUG
+#define TARA_DCHECK(cond, status) ((cond) ? true : (atomicOr((status), 2), false))
+#define TARA_DCHECK_RECORD(cond, status) \
+  do {                                   \
+    if (!(cond)) atomicOr((status), 2);  \
+  } while (0)
+#else
+#define TARA_DCHECK(cond, status) true
+#define TARA_DCHECK_RECORD(cond, status) ((void)0)
+#endif
+
 // The rule's parameters prepared on the host (double precision, then rounded once).
 struct BiasParams {
   float window;        // free window (s)

@@ -14,7 +14,8 @@ namespace tara {
 __global__ void __launch_bounds__(128)
 tile_summary_kernel(const uint8_t* __restrict__ seg, const float* __restrict__ time_s,
                     const uint8_t* __restrict__ pic, int N, long long batch_stride, int ntiles,
-                    BiasParams bp, TileRec* __restrict__ recs, float4* __restrict__ keyinfo) {
+                    BiasParams bp, TileRec* __restrict__ recs, float4* __restrict__ keyinfo,
+                    int* status) {
   const int tile = blockIdx.x;
   const int set = blockIdx.y;
   const int t = threadIdx.x;
@@ -29,6 +30,8 @@ tile_summary_kernel(const uint8_t* __restrict__ seg, const float* __restrict__ t
     s = seg[base + tok];
     tm = time_s[base + tok];
     pc = pic[base + tok];
+    // debug build: the clock of every target and guide token is a finite number
+    TARA_DCHECK_RECORD(!(s == kSegTarget || s == kSegGuide) || isfinite(tm), status);
   }
   const float inf = __int_as_float(0x7f800000);
   float tq_lo = (valid && s == kSegTarget) ? tm : inf;
