@@ -172,6 +172,13 @@ def test_rejects_shape(lib):
                  meta=_meta(N=0)) == -2
 
 
+def test_rejects_more_work_items_than_an_int_holds(lib):
+    # 46,340 x 46,340 planes fit the plane count, but with 1,024 tokens each (eight 128-token
+    # query tiles, two work items of four) the 4.3e9 work items do not fit an int
+    Q = _t(shape=(46340, 46340, 1024, 128))
+    assert _call(lib, Q=Q, K=Q, V=Q, O=Q, meta=_meta(N=1024)) == -11
+
+
 def test_rejects_head_dim(lib):
     for d in (32, 96, 256):
         s = (1, 2, 300, d)

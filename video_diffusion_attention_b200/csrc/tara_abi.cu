@@ -326,6 +326,9 @@ int validate(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
   }
   if (Q->B > 65535 || Q->H > 65535) return TARA_ERR_TOO_LARGE;
   if ((long long)Q->B * Q->H > 0x7fffffffLL) return TARA_ERR_TOO_LARGE;
+  // the persistent kernel numbers its work items (planes x groups of four query tiles) in int
+  if ((long long)Q->B * Q->H * ((((long long)Q->N + kTile - 1) / kTile + 3) / 4) > 0x7fffffffLL)
+    return TARA_ERR_TOO_LARGE;
   for (const tara_tensor* t : ts)
     if (!aligned16(t->ptr)) return TARA_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(LSE) & 3u) != 0) return TARA_ERR_ALIGN;
