@@ -154,8 +154,10 @@ const char* tara_status_string(int status);
 /* ---- the forward pass ------------------------------------------------------------------ */
 /* Computes O and LSE as defined at the top of this file.
  *   Q, K, V : device tensors [B][H][N][D], same shape and dtype.  bf16/fp16 run on the
- *             tensor-core kernel (D = 64 or 128); fp32 runs on the exact CUDA-core kernel
- *             (any D from 1 to 256).  Base pointers 16-byte aligned.
+ *             tensor-core kernels (D = 128: a persistent kernel on SM pairs, one cluster of
+ *             two CTAs per two SMs walking (branch, head, four-query-tile) work items; D = 64
+ *             and 8-bit Q K^T: one CTA per two query tiles); fp32 runs on the exact CUDA-core
+ *             kernel (any D from 1 to 256).  Base pointers 16-byte aligned.
  *   meta    : per-token metadata (device pointers), meta->N == N.
  *   p       : rule parameters (host pointer, read during the call only).
  *   O       : device tensor [B][H][N][D] of the same dtype (written).
@@ -164,7 +166,8 @@ const char* tara_status_string(int status);
  * Every O row and LSE entry is written; no other memory of the caller is touched.
  * Extra bindings: 0..3; their gains follow the same domain; extra_m must be non-NULL and
  * 4-byte aligned when there are any, and extra_m_stride at least the length of one m array.
- * Errors: TARA_ERR_NULL, _SHAPE, _DTYPE, _HEAD_DIM, _PARAM, _ALIGN, _TOO_LARGE (checked
+ * Errors: TARA_ERR_NULL, _SHAPE, _DTYPE, _HEAD_DIM, _PARAM, _ALIGN, _TOO_LARGE (B or H
+ * above 65535, B*H or the work items B*H*ceil(ceil(N/128)/4) above 2^31-1; all checked
  * before any launch), TARA_ERR_CUDA (workspace allocation or launch failure).             */
 int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
                       const tara_token_meta* meta, const tara_params* p,
