@@ -221,11 +221,12 @@ int tara_quantize_qk_int8(const tara_tensor* Q, const tara_tensor* K, int8_t* q_
                           float* q_scale, int8_t* k_codes, float* k_scale, void* stream);
 
 /* ---- allocation-free variant ------------------------------------------------------------ */
-/* Largest scratch (bytes) tara_attn_forward_noalloc can use: per metadata set, 16 bytes per
- * token plus 32 bytes per 128-token tile (4 MiB covers one shared set of up to ~260,000
+/* Largest scratch (bytes) tara_attn_forward_noalloc can use: per metadata set and 128-token
+ * tile, two copies (ascending and descending tile order) of a 32-byte tile record and of
+ * 128 16-byte key records, 4,160 bytes (8 MiB covers one shared set of up to ~258,000
  * tokens).  The array is part of the loaded module: every device that loads the library
  * holds it until the process exits.                                                       */
-#define TARA_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define TARA_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /* Same operation, arguments and checks as tara_attn_forward for bf16/fp16 inputs, but it
  * never allocates: no cudaMalloc, no cudaFree, no allocating library call.  It is meant for

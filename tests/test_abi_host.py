@@ -102,15 +102,17 @@ def _call_noalloc(lib, Q, meta, p=None):
 
 
 def _noalloc_scratch(nsets, N):
-    """Bytes of scratch the allocation-free entry point needs: per metadata set a 32-byte
-    record per 128-token tile and a 16-byte record per token, each part rounded to 256."""
+    """Bytes of scratch the allocation-free entry point needs: per metadata set and 128-token
+    tile, in ascending and in descending tile order, a 32-byte tile record and 128 16-byte key
+    records; each of the two arrays rounded to 256 bytes."""
     up = lambda x: (x + 255) // 256 * 256
-    return up(nsets * ((N + 127) // 128) * 32) + up(nsets * N * 16)
+    ntiles = (N + 127) // 128
+    return up(2 * nsets * ntiles * 32) + up(2 * nsets * ntiles * 128 * 16)
 
 
 def _noalloc_max_tokens(nsets):
     cap = B.TARA_NOALLOC_SCRATCH_BYTES
-    N = cap // (16 * nsets)
+    N = cap // (32 * nsets) + 128
     while _noalloc_scratch(nsets, N) > cap:
         N -= 1
     return N
@@ -120,8 +122,8 @@ def _noalloc_max_tokens(nsets):
 def test_noalloc_rejects_sizes_above_its_scratch(lib, nsets):
     # one token more than the fixed array holds is refused before any CUDA call
     header = open(os.path.join(ROOT, "include", "tara_attn.h")).read()
-    assert "#define TARA_NOALLOC_SCRATCH_BYTES (4u << 20)" in header
-    assert B.TARA_NOALLOC_SCRATCH_BYTES == 4 << 20
+    assert "#define TARA_NOALLOC_SCRATCH_BYTES (8u << 20)" in header
+    assert B.TARA_NOALLOC_SCRATCH_BYTES == 8 << 20
     n_fit = _noalloc_max_tokens(nsets)
     n = n_fit + 1
     assert _noalloc_scratch(nsets, n) > B.TARA_NOALLOC_SCRATCH_BYTES

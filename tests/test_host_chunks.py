@@ -21,7 +21,7 @@ size_t forward_workspace_bytes(const tara_tensor*, const tara_token_meta*, const
 }
 int forward_with_workspace(const tara_tensor*, const tara_tensor*, const tara_tensor*,
                            const tara_token_meta*, const tara_params*, tara_tensor*, float*,
-                           void*, size_t, void*) {
+                           void*, size_t, void*, long long) {
   return TARA_ERR_CUDA;
 }
 }  // namespace tara

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libtara_attn.so")
 
 TARA_BF16, TARA_FP16, TARA_FP32 = 0, 1, 2
 # size of the fixed scratch array of tara_attn_forward_noalloc (the header's define)
-TARA_NOALLOC_SCRATCH_BYTES = 4 << 20
+TARA_NOALLOC_SCRATCH_BYTES = 8 << 20
 SEG_TEXT, SEG_PICTURE, SEG_TARGET, SEG_GUIDE, SEG_AUDIO, SEG_OTHER_VIDEO = range(6)
 
 STATUS = {

@@ -5,8 +5,11 @@
 // items c, c + G, c + 2G, ... (G clusters) in head-major order.  An item is four 128-row query
 // tiles of one (branch, head): CTA r of the pair holds tiles 4q + 2t + r for t = 0, 1.  All
 // clusters start their n-th item at about the same time and stream the same head's K and V in
-// near lockstep, so a head's keys and values are read from DRAM about once and then served
-// from L2 to every cluster (a grid of one CTA pair per item let later waves re-read them).
+// near lockstep, so a head's keys and values are read from DRAM about once per round of items
+// and then served from L2 to every cluster (a grid of one CTA pair per item let later waves
+// re-read them).  Consecutive rounds walk the key tiles in opposite directions: a round starts
+// on the tiles the round before read last, which L2 still holds, instead of on the tiles it
+// read first, which a head's 55 MB of K and V (at 107k tokens) has pushed out by then.
 // The even CTA issues every MMA with
 // cta_group::2, M = 256: MMA "t" covers tile t of both CTAs.  Each CTA supplies its own 128 rows
 // of the A operand (Q for S = Q K^T, P for O += P V) and half of every B operand: keys
@@ -112,7 +115,12 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int first_item = (int)(blockIdx.x >> 1);
   // Every role walks the same items in the same order.  Barrier phases run on across items:
   // the g-th key tile this cluster processes (g = item ordinal * nk + j) completes phase g of
-  // the per-tile barriers, and ring slot s holds K or V half-tile number 2g or 2g + 1.
+  // the per-tile barriers, and ring slot s holds K or V half-tile number 2g or 2g + 1.  Step j
+  // of an item processes key tile j, or nk - 1 - j on items that walk the keys descending (the
+  // order changes the softmax's result by rounding only).
+  auto descending = [&](int item) -> bool {
+    return (((uint32_t)(args.item_base + item)) / (uint32_t)args.order_span) & 1u;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -176,6 +184,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       for (int item = first_item, k = 0; ok && item < n_items; item += n_clusters, ++k) {
         const int bh = item / groups;
         const int qt_base = (item - bh * groups) * kPairTiles + (int)rank;
+        const bool desc = descending(item);
         // Q of the previous item is read by its last QK^T
         if (k > 0 && !(ok = mbar_wait(q_empty, (uint32_t)(k - 1) & 1u, abort_flag, kWaitLimitNs))) break;
         if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * S::kQTileBytes);
@@ -190,7 +199,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           if (leader) mbar_arrive_expect_tx(&kv_full[slot], 2 * HB);
           const uint32_t full_l = mapa_shared(smem_u32(&kv_full[slot]), 0);
           uint8_t* dst = sKV + slot * HB;
-          const int j = h2 >> 1;
+          const int j = desc ? nk - 1 - (h2 >> 1) : h2 >> 1;
           if ((h2 & 1) == 0) {
             // K_j rows [64r, 64r + 64): two 64-row x 128-byte panels (head-dim halves)
             for (int p = 0; p < 2; ++p)
@@ -320,8 +329,12 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const bool row_ok = (qtile < args.ntiles) && (row < N);
       const int mset = args.per_branch_meta ? bh / args.H : 0;
       const long long mtok = (long long)mset * args.meta_stride;
-      const TileRec* recs = args.recs + (long long)mset * args.ntiles;
-      const float4* kinfo = args.keyinfo + (long long)mset * N;
+      // the records in the order this item walks the keys: step j reads tile record j and key
+      // records [128 j, 128 j + 128) of the ascending or the descending copy
+      const bool desc = descending(item);
+      const TileRec* krecs = (desc ? args.recs_desc : args.recs) + (long long)mset * args.ntiles;
+      const float4* kinfo =
+          (desc ? args.keyinfo_desc : args.keyinfo) + (long long)mset * args.ntiles * kTile;
 
       bool is_tgt = false;
       float t_q = 0.0f, m_q = 0.0f;
@@ -347,7 +360,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       TileRec qr;
       if (qtile < args.ntiles) {
-        qr = recs[qtile];
+        qr = args.recs[(long long)mset * args.ntiles + qtile];   // ascending copy: tile qtile
       } else {
         qr.segmask = 0;
         qr.picmask = 0;
@@ -358,11 +371,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       float m_run = ninf, l_run = 0.0f;
 
-      TileRec kr_next = recs[0];
+      TileRec kr_next = krecs[0];
       for (int j = 0; j < nk; ++j) {
         const int gj = g + j;
         const TileRec kr = kr_next;
-        if (j + 1 < nk) kr_next = recs[j + 1];   // in flight while this tile is processed
+        if (j + 1 < nk) kr_next = krecs[j + 1];   // in flight while this tile is processed
         const float sl = bp.scale_log2;
         float cval;
         const int cls = classify_pair(qr, kr, bp, &cval);
@@ -378,8 +391,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           // stage the tile's key records in shared memory (one coalesced load per thread);
           // two buffers, so a warp one iteration ahead never overwrites records another warp
           // of the group still reads
-          const int key = j * kTile + r;
-          kb[r] = key < N ? kinfo[key] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          kb[r] = kinfo[j * kTile + r];   // zero records past the sequence's end
           if (!(ok = warp_rendezvous(&stage_bar[t], stage_phase, abort_flag, kWaitLimitNs))) break;
         }
         if (!(ok = warp_wait(&s_full[t], (uint32_t)gj & 1u, abort_flag, kWaitLimitNs))) break;

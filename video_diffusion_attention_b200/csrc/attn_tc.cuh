@@ -75,8 +75,13 @@ struct TcArgs {
   const uint8_t* seg;
   const float* time_s;
   const float* m;
+  // Records written by the tile-summary kernel, per metadata set: ntiles tile records and
+  // ntiles * 128 key records (zero past the sequence's end), in ascending tile order; the
+  // *_desc copies hold the same records with the tile order reversed (tile ntiles - 1 first)
   const TileRec* recs;
   const float4* keyinfo;
+  const TileRec* recs_desc;
+  const float4* keyinfo_desc;
   long long meta_stride;   // tokens between metadata sets (0: one set for all branches)
   int N, H, ntiles;
   int B;                   // branches (the persistent kernel walks all B x H planes)
@@ -86,6 +91,12 @@ struct TcArgs {
   ExtraMasks xm;           // masks of chained bindings beyond the first (bp.n_extra of them)
   const float* q_scale;    // INT8 QK^T: per-token Q scales [B*H][N]
   const float* k_scale;    // INT8 QK^T: per-key-tile K scales [B*H][ntiles]
+  // SM-pair kernel: work item i of this call is item item_base + i of the larger call its
+  // planes were cut from (item_base 0 for an uncut call); it walks the keys ascending when
+  // ((item_base + i) / order_span) is even, descending when it is odd
+  long long plane_base;    // host side: index of this call's plane 0 in the larger call
+  int item_base;
+  int order_span;
 };
 
 // A wait every lane of the warp leaves together (the tcgen05 loads and stores that follow are
@@ -357,7 +368,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int mset = args.per_branch_meta ? blockIdx.z : 0;
     const long long mtok = (long long)mset * args.meta_stride;
     const TileRec* recs = args.recs + (long long)mset * args.ntiles;
-    const float4* kinfo = args.keyinfo + (long long)mset * N;
+    const float4* kinfo = args.keyinfo + (long long)mset * args.ntiles * kTile;
 
     bool is_tgt = false;
     float t_q = 0.0f, m_q = 0.0f;

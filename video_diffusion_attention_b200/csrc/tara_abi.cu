@@ -270,8 +270,17 @@ int launch_pair(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V
   const long long items = (long long)B * H * ((ntiles + kPairTiles - 1) / kPairTiles);
   const long long clusters = std::min<long long>(items, std::max(1, sms / 2));
   dim3 grid((unsigned)(2 * clusters), 1, 1);
+  // the key order flips every (SMs / 2) items: with a full grid, every round of concurrent
+  // items walks the keys the opposite way to the round before and starts on the key tiles
+  // that round read last, which are still in L2.  The span depends on the device only, so a
+  // plane's result does not depend on how many planes share the call.
+  const long long item_base = a.plane_base * ((ntiles + kPairTiles - 1) / kPairTiles);
+  if (item_base + items > 0x7fffffffLL) return TARA_ERR_TOO_LARGE;
+  TcArgs ap = a;
+  ap.item_base = (int)item_base;
+  ap.order_span = std::max(1, sms / 2);
   if (record_start(stream) != TARA_OK) return TARA_ERR_CUDA;
-  attn_pair_kernel<kBF16><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, a);
+  attn_pair_kernel<kBF16><<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, ap);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
   return record_stop(stream);
 }
@@ -288,6 +297,9 @@ TcArgs make_tc_args(const tara_token_meta* meta, tara_tensor* O, float* LSE, Til
   a.m = meta->m;
   a.recs = recs;
   a.keyinfo = keyinfo;
+  const long long nsets = meta->batch_stride != 0 ? O->B : 1;
+  a.recs_desc = recs + nsets * ntiles;
+  a.keyinfo_desc = keyinfo + nsets * ntiles * kTile;
   a.meta_stride = (long long)meta->batch_stride;
   a.N = N;
   a.H = H;
@@ -299,6 +311,9 @@ TcArgs make_tc_args(const tara_token_meta* meta, tara_tensor* O, float* LSE, Til
   a.xm = ExtraMasks{meta->extra_m, (long long)meta->extra_m_stride};
   a.q_scale = q_scale;
   a.k_scale = k_scale;
+  a.plane_base = 0;
+  a.item_base = 0;
+  a.order_span = 1;
   return a;
 }
 
@@ -352,7 +367,8 @@ int validate(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
 }
 
 // Workspace of one tensor-core forward call: tile records and per-key records of every
-// metadata set, then (qk_int8 only) the 8-bit copies of Q and K and their scales.
+// metadata set, in ascending and in descending tile order (tile_summary.cuh), then (qk_int8
+// only) the 8-bit copies of Q and K and their scales.
 struct WsLayout {
   int nsets;
   size_t rec, key, code, qs, ks, total;
@@ -363,8 +379,8 @@ WsLayout ws_layout(const tara_tensor* Q, const tara_token_meta* meta, const tara
   const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
   const int ntiles = (N + kTile - 1) / kTile;
   L.nsets = meta->batch_stride != 0 ? B : 1;
-  L.rec = round_up((size_t)L.nsets * ntiles * sizeof(TileRec), 256);
-  L.key = round_up((size_t)L.nsets * N * sizeof(float4), 256);
+  L.rec = round_up(2 * (size_t)L.nsets * ntiles * sizeof(TileRec), 256);
+  L.key = round_up(2 * (size_t)L.nsets * ntiles * kTile * sizeof(float4), 256);
   const bool q8 = p->qk_int8 != 0;
   L.code = q8 ? round_up((size_t)B * H * N * D, 256) : 0;
   L.qs = q8 ? round_up((size_t)B * H * N * sizeof(float), 256) : 0;
@@ -376,9 +392,10 @@ WsLayout ws_layout(const tara_tensor* Q, const tara_token_meta* meta, const tara
 // The forward pass after argument checks, with g_mu held.  ws_ext == nullptr: the device's
 // shared workspace, ordered against every other call through ws_free.  Otherwise the caller's
 // workspace of ws_ext_bytes (at least ws_layout(...).total of the shape), which the caller orders.
+// plane_base: index of plane 0 within a larger call these planes were cut from (0 otherwise).
 int forward_locked(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
                    const tara_token_meta* meta, const tara_params* p, tara_tensor* O, float* LSE,
-                   cudaStream_t stream, void* ws_ext, size_t ws_ext_bytes) {
+                   cudaStream_t stream, void* ws_ext, size_t ws_ext_bytes, long long plane_base) {
   int rc = TARA_OK;
   const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
   const BiasParams bp = make_bias_params(p, D);
@@ -448,7 +465,8 @@ int forward_locked(const tara_tensor* Q, const tara_tensor* K, const tara_tensor
       keyinfo, st->status);
   if (cudaGetLastError() != cudaSuccess) return TARA_ERR_CUDA;
 
-  const TcArgs a = make_tc_args(meta, O, LSE, recs, keyinfo, N, H, ntiles, st->status, bp, qs, ks);
+  TcArgs a = make_tc_args(meta, O, LSE, recs, keyinfo, N, H, ntiles, st->status, bp, qs, ks);
+  a.plane_base = plane_base;
   const bool bf16 = Q->dtype == TARA_BF16;
   if (q8)
     rc = bf16 ? launch_tc<true, 128, true>(mq, mk, mv, a, B, H, ntiles, stream, st)
@@ -473,13 +491,16 @@ size_t forward_workspace_bytes(const tara_tensor* Q, const tara_token_meta* meta
 
 int forward_with_workspace(const tara_tensor* Q, const tara_tensor* K, const tara_tensor* V,
                            const tara_token_meta* meta, const tara_params* p, tara_tensor* O,
-                           float* LSE, void* ws, size_t ws_bytes, void* stream) {
+                           float* LSE, void* ws, size_t ws_bytes, void* stream,
+                           long long plane_base) {
   int rc = validate(Q, K, V, meta, p, O, LSE);
+  if (plane_base < 0) return TARA_ERR_SHAPE;
   if (rc != TARA_OK) return rc;
   if (Q->dtype != TARA_FP32 && !ws) return TARA_ERR_NULL;
   if (!aligned16(ws)) return TARA_ERR_ALIGN;
   std::lock_guard<std::mutex> lock(g_mu);
-  return forward_locked(Q, K, V, meta, p, O, LSE, static_cast<cudaStream_t>(stream), ws, ws_bytes);
+  return forward_locked(Q, K, V, meta, p, O, LSE, static_cast<cudaStream_t>(stream), ws, ws_bytes,
+                        plane_base);
 }
 
 }  // namespace tara
@@ -528,7 +549,7 @@ int tara_attn_forward(const tara_tensor* Q, const tara_tensor* K, const tara_ten
   int rc = validate(Q, K, V, meta, p, O, LSE);
   if (rc != TARA_OK) return rc;
   std::lock_guard<std::mutex> lock(g_mu);
-  return forward_locked(Q, K, V, meta, p, O, LSE, static_cast<cudaStream_t>(stream_), nullptr, 0);
+  return forward_locked(Q, K, V, meta, p, O, LSE, static_cast<cudaStream_t>(stream_), nullptr, 0, 0);
 }
 
 int tara_quantize_qk_int8(const tara_tensor* Q, const tara_tensor* K, int8_t* q_codes,
@@ -699,8 +720,9 @@ extern "C" int tara_attn_forward_noalloc(const tara_tensor* Q, const tara_tensor
   const int B = Q->B, H = Q->H, N = Q->N, D = Q->D;
   const int ntiles = (N + kTile - 1) / kTile;
   const size_t nsets = meta->batch_stride != 0 ? (size_t)B : 1;
-  const size_t rec_bytes = round_up(nsets * (size_t)ntiles * sizeof(TileRec), 256);
-  const size_t key_bytes = round_up(nsets * (size_t)N * sizeof(float4), 256);
+  // the ascending and the descending copy of every record (tile_summary.cuh)
+  const size_t rec_bytes = round_up(2 * nsets * (size_t)ntiles * sizeof(TileRec), 256);
+  const size_t key_bytes = round_up(2 * nsets * (size_t)ntiles * kTile * sizeof(float4), 256);
   if (rec_bytes + key_bytes > kStaticScratchBytes) return TARA_ERR_TOO_LARGE;
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);

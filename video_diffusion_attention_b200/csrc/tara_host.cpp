@@ -237,7 +237,7 @@ extern "C" int tara_attn_forward_host(const tara_tensor* Q, const tara_tensor* K
       dm.m = reinterpret_cast<const float*>(base + off_m) + mo;
       dm.extra_m = nx > 0 ? reinterpret_cast<const float*>(base + off_x) + mo : nullptr;
       dm.batch_stride = 0;
-      rc = tara::forward_with_workspace(&tq, &tk, &tv, &dm, p, &to, dl, dws, ws_bytes, comp);
+      rc = tara::forward_with_workspace(&tq, &tk, &tv, &dm, p, &to, dl, dws, ws_bytes, comp, p0);
       if (rc != TARA_OK) break;
       cuda_ok = cudaEventRecord(pipe.ev_comp[k], comp) == cudaSuccess &&
                 cudaStreamWaitEvent(pipe.s_out, pipe.ev_comp[k], 0) == cudaSuccess &&

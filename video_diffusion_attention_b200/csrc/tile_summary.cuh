@@ -5,6 +5,13 @@
 // TARGET and GUIDE tokens with warp shuffles, then combines the four warps in shared memory.
 // The attention kernels classify every (query tile, key tile) pair from two of these records
 // instead of evaluating the bias on every edge.
+//
+// Layout (nsets = gridDim.y metadata sets): recs[set * ntiles + tile] and
+// keyinfo[set * ntiles * 128 + tok] in ascending tile order, the key records past the
+// sequence's end zero; then the same records with the tile order reversed, at
+// recs[(nsets + set) * ntiles + ntiles - 1 - tile] and
+// keyinfo[(nsets + set) * ntiles * 128 + (ntiles - 1 - tile) * 128 + t], for work that walks
+// the keys from the last tile to the first.
 #pragma once
 
 #include "tara_common.cuh"
@@ -43,17 +50,20 @@ tile_summary_kernel(const uint8_t* __restrict__ seg, const float* __restrict__ t
   // all-same-picture test: every valid token PICTURE with the same index
   uint32_t pic_or_any = (valid && s == kSegPicture) ? pc : 0xFFu;
 
-  // per-key record (the key side of the bias)
-  if (valid) {
+  // per-key record (the key side of the bias); zero for positions past the end
+  const int nsets = (int)gridDim.y;
+  const long long kstride = (long long)ntiles * kTile;
+  {
     float4 rec = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (s == kSegGuide) {
+    if (valid && s == kSegGuide) {
       rec.x = tm;
       rec.z = 1.0f;
-    } else if (s == kSegPicture && pc < 16 && ((bp.lng_nz >> pc) & 1u)) {
+    } else if (valid && s == kSegPicture && pc < 16 && ((bp.lng_nz >> pc) & 1u)) {
       rec.y = bp.lng[pc];
       rec.w = (float)pc;
     }
-    keyinfo[(long long)set * N + tok] = rec;
+    keyinfo[(long long)set * kstride + tok] = rec;
+    keyinfo[(long long)(nsets + set) * kstride + (long long)(ntiles - 1 - tile) * kTile + t] = rec;
   }
 
 #pragma unroll
@@ -96,6 +106,7 @@ tile_summary_kernel(const uint8_t* __restrict__ seg, const float* __restrict__ t
     r.nvalid = sh_u[0][4] + sh_u[1][4] + sh_u[2][4] + sh_u[3][4];
     r.single_pic = (r.segmask == (1u << kSegPicture) && lo == hi && lo >= 1 && lo <= 9) ? lo : 0u;
     recs[(long long)set * ntiles + tile] = r;
+    recs[(long long)(nsets + set) * ntiles + (ntiles - 1 - tile)] = r;
   }
 }
 
