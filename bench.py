@@ -62,7 +62,9 @@ def load_peaks():
 
 
 # the device sources the attention kernel is compiled from
-KERNEL_SOURCES = ("attn_pair.cuh", "attn_tc.cuh", "sm100_ptx.cuh", "tara_common.cuh")
+# (the tile-summary kernel lays out the records the attention kernels read)
+KERNEL_SOURCES = ("attn_pair.cuh", "attn_tc.cuh", "sm100_ptx.cuh", "tara_common.cuh",
+                  "tile_summary.cuh")
 
 
 def kernel_source_hash() -> str:
