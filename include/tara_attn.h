@@ -32,7 +32,8 @@
  *     entry point exits, throws or prints.
  *   - Ownership: the caller owns every buffer.  Device buffers are never freed or retained by
  *     the library beyond the call.  tara_attn_forward keeps one internal per-device workspace
- *     (per metadata set 16 bytes per token plus 32 bytes per 128-token tile; with qk_int8,
+ *     (per metadata set and 128-token tile 4,160 bytes: tile and per-key records, each in
+ *     ascending and in descending tile order; with qk_int8,
  *     also 2*B*H*N*D bytes of codes and 4*B*H*(N + N/128) bytes of scales); it is allocated
  *     with cudaMalloc the first time a device sees a given size and reused afterwards, so the
  *     first call on a device (or with a larger size) must not be made while a stream is being
