@@ -32,11 +32,14 @@
 //   warp 10    in the even CTA, one thread issues the PV stream: PV_t(j) once P_t(j) is
 //              written and V_j has landed (two issuers: a single thread issuing both streams
 //              in turn left the tensor pipe idle between MMA groups)
-//   warp 11    idle (completes the third warpgroup for the register split)
+//   warp 11    one thread classifies the (query tile, key tile) pairs ahead of the softmax
+//              (tara_common.cuh: zero, constant, per-row or per-edge bias) into a ring of
+//              shared-memory entries, so the softmax warps read one entry per key tile
+//              instead of loading two tile summaries and classifying them
 //
-// Per key tile and query tile the softmax: waits for S, loads the whole row (one 128-column
-// tcgen05.ld), tells the issuer that S may be overwritten, applies the tile class's bias
-// (tara_common.cuh), takes the row max, computes all 128 exponentials into packed 16-bit
+// Per key tile and query tile the softmax: reads the tile pair's class, waits for S, loads the
+// whole row (one 128-column tcgen05.ld), tells the issuer that S may be overwritten, applies
+// the class's bias, takes the row max, computes all 128 exponentials into packed 16-bit
 // registers, then waits for the previous PV of its tile (the P buffer's last reader; usually
 // long done by then), stores P, rescales the O row if the running max grew by more than 2^8,
 // and signals P ready.  Every wait is bounded; a CTA that gives up sets an abort flag, the pair
@@ -59,10 +62,12 @@ struct PairShape {
   static constexpr int kPTileBytes = kTile * kTile * 2;   // 32 KB: P of one query tile
   static constexpr int kKeyBufBytes = 2 * 2 * kTile * 16; // [query tile][parity][key] float4
   static constexpr int kRowWBytes = 2 * kTile * 17 * 4;   // [tile][row] extra-binding weights
-  static constexpr int kBarCount = 2 + 2 * kStages + 2 * 4 + 2 + 1 + 2 + 8;
+  static constexpr int kClsRing = 8;                      // classification ring slots
+  static constexpr int kClsBytes = kClsRing * 2 * 8;      // [slot][query tile] uint2
+  static constexpr int kBarCount = 2 + 2 * kStages + 2 * 4 + 2 + 1 + 2 + 8 + 2 * kClsRing;
   static constexpr int kSmemBytes = 1024 /*alignment slack*/ + 2 * kQTileBytes +
                                     kStages * kHalfBytes + 2 * kPTileBytes + kKeyBufBytes +
-                                    kRowWBytes + kBarCount * 8 + 16;
+                                    kRowWBytes + kClsBytes + kBarCount * 8 + 16;
   static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
   static constexpr uint32_t kColO = 256;                  // O_t at kColO + 128 t
 };
@@ -87,7 +92,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint8_t* sP = sKV + NS * HB;                          // 2 tiles
   float4* kbuf = reinterpret_cast<float4*>(sP + 2 * S::kPTileBytes);
   float* rowx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(kbuf) + S::kKeyBufBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(rowx) + S::kRowWBytes);
+  uint2* cls_ring = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(rowx) + S::kRowWBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(cls_ring) + S::kClsBytes);
   uint64_t* q_full = bars;              // even CTA: Q of both CTAs landed
   uint64_t* q_empty = q_full + 1;       // both CTAs (2-SM commit): the last QK^T of an item read Q
   uint64_t* kv_full = q_empty + 1;      // even CTA: both halves of slot s landed
@@ -100,7 +106,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint64_t* exit_bar = drain + 2;       // the peer is done with this CTA's memory
   uint64_t* stage_bar = exit_bar + 1;   // [2] per query tile: the 4 warps of its group
   uint64_t* exp_tok = stage_bar + 2;    // [lane quarter][tile]: that warp may run its exponentials
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(exp_tok + 8);
+  uint64_t* cls_full = exp_tok + 8;     // [slot] the classifier wrote both tiles' entries
+  uint64_t* cls_empty = cls_full + S::kClsRing;   // [slot] the 8 softmax warps have read them
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cls_empty + S::kClsRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,6 +148,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(&exp_tok[2 * q], 1);
       mbar_init(&exp_tok[2 * q + 1], 1);
       mbar_arrive(&exp_tok[2 * q]);   // tile 0 goes first
+    }
+    for (int c = 0; c < S::kClsRing; ++c) {
+      mbar_init(&cls_full[c], 1);
+      mbar_init(&cls_empty[c], 8);
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
@@ -298,6 +310,56 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       umma_commit_pair(my_drain);
       volatile int no_abort = 0;
       mbar_wait(my_drain, 0, &no_abort, kDrainLimitNs);
+    } else if (warp == 11 && lane == 0) {
+      // ------------------------------ tile-pair classifier (both CTAs) -----------------
+      // Runs up to kClsRing key tiles ahead of the softmax warps: for step g of the walk it
+      // classifies (query tile t of this CTA, the step's key tile) for t = 0, 1 and writes
+      // {class | Picture index << 8 | valid keys << 16, parameter} to ring slot g % kClsRing,
+      // the parameter being the constant bias (natural units) of the constant classes and
+      // the guide frame's time of a single-frame guide tile.
+      const BiasParams& bp = args.bp;
+      bool ok = true;
+      int g = 0;
+      for (int item = first_item; ok && item < n_items; item += n_clusters, g += nk) {
+        const int bh = item / groups;
+        const int mset = args.per_branch_meta ? bh / args.H : 0;
+        const TileRec* qrecs = args.recs + (long long)mset * args.ntiles;
+        const TileRec* krecs =
+            (descending(item) ? args.recs_desc : args.recs) + (long long)mset * args.ntiles;
+        TileRec qr[2];
+        for (int t = 0; t < 2; ++t) {
+          const int qtile = (item - bh * groups) * kPairTiles + (int)rank + 2 * t;
+          if (qtile < args.ntiles) {
+            qr[t] = qrecs[qtile];
+          } else {
+            qr[t].segmask = 0;   // no rows: classified as unbiased
+            qr[t].picmask = 0;
+            qr[t].nvalid = 0;
+            qr[t].single_pic = 0;
+            qr[t].tq_min = qr[t].tk_min = 0.0f;
+            qr[t].tq_max = qr[t].tk_max = 0.0f;
+          }
+        }
+        TileRec kr_next = krecs[0];
+        for (int j = 0; j < nk; ++j) {
+          const int gj = g + j;
+          const int slot = gj & (S::kClsRing - 1);
+          const TileRec kr = kr_next;
+          if (j + 1 < nk) kr_next = krecs[j + 1];
+          if (!(ok = mbar_wait(&cls_empty[slot], ((uint32_t)(gj / S::kClsRing) & 1u) ^ 1u,
+                               abort_flag, kWaitLimitNs)))
+            break;
+          for (int t = 0; t < 2; ++t) {
+            float cval;
+            const int cls = classify_pair(qr[t], kr, bp, &cval);
+            const float par = cls == kClsRowGuide ? kr.tk_min : cval;
+            cls_ring[slot * 2 + t] =
+                make_uint2((uint32_t)cls | ((kr.single_pic & 15u) << 8) | (kr.nvalid << 16),
+                           __float_as_uint(par));
+          }
+          mbar_arrive(&cls_full[slot]);
+        }
+      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kTcSoftmaxRegs) : "memory");
@@ -329,12 +391,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const bool row_ok = (qtile < args.ntiles) && (row < N);
       const int mset = args.per_branch_meta ? bh / args.H : 0;
       const long long mtok = (long long)mset * args.meta_stride;
-      // the records in the order this item walks the keys: step j reads tile record j and key
-      // records [128 j, 128 j + 128) of the ascending or the descending copy
-      const bool desc = descending(item);
-      const TileRec* krecs = (desc ? args.recs_desc : args.recs) + (long long)mset * args.ntiles;
-      const float4* kinfo =
-          (desc ? args.keyinfo_desc : args.keyinfo) + (long long)mset * args.ntiles * kTile;
+      // the key records in the order this item walks the keys: step j reads records
+      // [128 j, 128 j + 128) of the ascending or the descending copy
+      const float4* kinfo = (descending(item) ? args.keyinfo_desc : args.keyinfo) +
+                            (long long)mset * args.ntiles * kTile;
 
       bool is_tgt = false;
       float t_q = 0.0f, m_q = 0.0f;
@@ -358,33 +418,27 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           wx[pidx] = acc;
         }
       }
-      TileRec qr;
-      if (qtile < args.ntiles) {
-        qr = args.recs[(long long)mset * args.ntiles + qtile];   // ascending copy: tile qtile
-      } else {
-        qr.segmask = 0;
-        qr.picmask = 0;
-        qr.nvalid = 0;
-        qr.single_pic = 0;
-        qr.tq_min = qr.tk_min = 0.0f;
-        qr.tq_max = qr.tk_max = 0.0f;
-      }
       float m_run = ninf, l_run = 0.0f;
 
-      TileRec kr_next = krecs[0];
       for (int j = 0; j < nk; ++j) {
         const int gj = g + j;
-        const TileRec kr = kr_next;
-        if (j + 1 < nk) kr_next = krecs[j + 1];   // in flight while this tile is processed
         const float sl = bp.scale_log2;
-        float cval;
-        const int cls = classify_pair(qr, kr, bp, &cval);
+        // this tile pair's class from the classifier warp (normally written long before)
+        const int cs = gj & (S::kClsRing - 1);
+        if (!(ok = warp_wait(&cls_full[cs], (uint32_t)(gj / S::kClsRing) & 1u, abort_flag,
+                             kWaitLimitNs)))
+          break;
+        const uint2 ce = cls_ring[cs * 2 + t];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cls_empty[cs]);
+        const int cls = (int)(ce.x & 0xffu);
+        const float cpar = __uint_as_float(ce.y);
         float rowb2 = 0.0f;
         if (is_tgt) {
-          if (cls == kClsConstCap) rowb2 = cval * kLog2e;
-          else if (cls == kClsRowGuide) rowb2 = -penalty_f32(fabsf(t_q - kr.tk_min), bp) * kLog2e;
+          if (cls == kClsConstCap) rowb2 = cpar * kLog2e;
+          else if (cls == kClsRowGuide) rowb2 = -penalty_f32(fabsf(t_q - cpar), bp) * kLog2e;
           else if (cls == kClsConstPic)
-            rowb2 = (bp.n_extra > 0 ? m_q * cval + wx[kr.single_pic & 15] : m_q * cval) * kLog2e;
+            rowb2 = (bp.n_extra > 0 ? m_q * cpar + wx[(ce.x >> 8) & 15u] : m_q * cpar) * kLog2e;
         }
         float4* kb = kbuf + (t * 2 + (gj & 1)) * kTile;
         if (cls == kClsFull) {
@@ -405,7 +459,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(s_free_l);
 
-        const int nv = (int)kr.nvalid;
+        const int nv = (int)(ce.x >> 16);
         if (nv < kTile) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
