@@ -61,18 +61,20 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-# the device sources the attention kernel is compiled from
-# (the tile-summary kernel lays out the records the attention kernels read)
+# the device sources each attention kernel is compiled from (the tile-summary kernel lays out
+# the records both read; the quantiser the 8-bit codes the INT8 kernel reads)
 KERNEL_SOURCES = ("attn_pair.cuh", "attn_tc.cuh", "sm100_ptx.cuh", "tara_common.cuh",
                   "tile_summary.cuh")
+KERNEL_SOURCES_INT8 = ("attn_tc.cuh", "quant_int8.cuh", "sm100_ptx.cuh", "tara_common.cuh",
+                       "tile_summary.cuh")
 
 
-def kernel_source_hash() -> str:
-    """sha256 (first 16 hex digits) of the kernel's device sources with // comments, trailing
+def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
+    """sha256 (first 16 hex digits) of a kernel's device sources with // comments, trailing
     blanks and empty lines removed: edits to comments leave it unchanged, edits to code do not."""
     import re
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources:
         with open(os.path.join(CSRC, f)) as fh:
             lines = (re.sub(r"//.*$", "", line).rstrip() for line in fh.read().splitlines())
             code = "\n".join(line for line in lines if line)
@@ -147,10 +149,14 @@ def recorded_traffic(workload: str):
             if "=" in line:
                 k, v = line.split("=", 1)
                 vals[k.strip()] = v.strip()
-    # a figure may carry its own source hash (taken on an earlier version of the same kernel)
+    # "<workload>_int8" figures belong to the INT8 kernel, the others to the 16-bit one; each
+    # kernel's figures carry the hash of its sources (kernel_source_sha256_16[_int8]), and a
+    # figure may carry its own (taken on an earlier version of the same kernel)
     key = "bytes_per_launch_" + workload
-    if vals.get("kernel_source_sha256_16_" + workload,
-                vals.get("kernel_source_sha256_16")) != kernel_source_hash():
+    int8 = workload.endswith("_int8")
+    default = vals.get("kernel_source_sha256_16_int8" if int8 else "kernel_source_sha256_16")
+    current = kernel_source_hash(KERNEL_SOURCES_INT8 if int8 else KERNEL_SOURCES)
+    if vals.get("kernel_source_sha256_16_" + workload, default) != current:
         return None
     return float(vals[key]) if key in vals else None
 

@@ -23,6 +23,7 @@ def test_traffic_needs_the_current_kernel_hash(tmp_path, monkeypatch):
 
 def test_a_figure_can_carry_its_own_hash(tmp_path, monkeypatch):
     h = bench.kernel_source_hash()
+    h8 = bench.kernel_source_hash(bench.KERNEL_SOURCES_INT8)
     monkeypatch.setattr(bench, "TRAFFIC_FILE", _write(tmp_path, (
         "kernel_source_sha256_16 = %s\n"
         "kernel_source_sha256_16_full_int8 = 0123456789abcdef\n"
@@ -32,9 +33,32 @@ def test_a_figure_can_carry_its_own_hash(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "TRAFFIC_FILE", _write(tmp_path, (
         "kernel_source_sha256_16 = 0123456789abcdef\n"
         "kernel_source_sha256_16_full_int8 = %s\n"
-        "bytes_per_launch_full = 10\nbytes_per_launch_full_int8 = 20\n" % h)))
+        "bytes_per_launch_full = 10\nbytes_per_launch_full_int8 = 20\n" % h8)))
     assert bench.recorded_traffic("full") is None
     assert bench.recorded_traffic("full_int8") == 20.0
+
+
+def test_each_kernel_has_its_own_source_hash(tmp_path, monkeypatch):
+    # a change to the pair kernel's source leaves the INT8 kernel's figures valid, and the
+    # reverse; a source both kernels read invalidates both
+    src = tmp_path / "csrc"
+    src.mkdir()
+    for f in set(bench.KERNEL_SOURCES) | set(bench.KERNEL_SOURCES_INT8):
+        (src / f).write_text("int %s = 1;\n" % f.split(".")[0])
+    monkeypatch.setattr(bench, "CSRC", str(src))
+    h, h8 = bench.kernel_source_hash(), bench.kernel_source_hash(bench.KERNEL_SOURCES_INT8)
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", _write(tmp_path, (
+        "kernel_source_sha256_16 = %s\nkernel_source_sha256_16_int8 = %s\n"
+        "bytes_per_launch_full = 10\nbytes_per_launch_full_int8 = 20\n" % (h, h8))))
+    assert bench.recorded_traffic("full") == 10.0 and bench.recorded_traffic("full_int8") == 20.0
+    (src / "attn_pair.cuh").write_text("int changed = 2;\n")
+    assert bench.recorded_traffic("full") is None and bench.recorded_traffic("full_int8") == 20.0
+    (src / "attn_pair.cuh").write_text("int attn_pair = 1;\n")
+    (src / "quant_int8.cuh").write_text("int changed = 2;\n")
+    assert bench.recorded_traffic("full") == 10.0 and bench.recorded_traffic("full_int8") is None
+    (src / "quant_int8.cuh").write_text("int quant_int8 = 1;\n")
+    (src / "tara_common.cuh").write_text("int changed = 2;\n")
+    assert bench.recorded_traffic("full") is None and bench.recorded_traffic("full_int8") is None
 
 
 def test_missing_file_reports_nothing(tmp_path, monkeypatch):
