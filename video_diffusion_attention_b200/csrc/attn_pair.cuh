@@ -10,11 +10,12 @@
 // re-read them).  Consecutive rounds walk the key tiles in opposite directions: a round starts
 // on the tiles the round before read last, which L2 still holds, instead of on the tiles it
 // read first, which a head's 55 MB of K and V (at 107k tokens) has pushed out by then.
-// The even CTA issues every MMA with
-// cta_group::2, M = 256: MMA "t" covers tile t of both CTAs.  Each CTA supplies its own 128 rows
-// of the A operand (Q for S = Q K^T, P for O += P V) and half of every B operand: keys
-// [64r, 64r + 64) of a key tile for QK^T and head-dim columns [64r, 64r + 64) of a value tile
-// for PV, so each SM loads and stores half of K and V.
+//
+// The even CTA issues every MMA with cta_group::2, M = 256: MMA "t" covers tile t of both
+// CTAs.  Each CTA supplies its own 128 rows of the A operand (Q for S = Q K^T, P for
+// O += P V) and half of every B operand: keys [64r, 64r + 64) of a key tile for QK^T and
+// head-dim columns [64r, 64r + 64) of a value tile for PV, so each SM loads and stores half
+// of K and V.
 //
 // Tensor memory of each CTA (512 columns): S_0 | S_1 | O_0 | O_1, fp32.  P_t (16-bit) is written
 // by the softmax threads to shared memory in the K-major 128-byte-swizzled layout the MMA reads
